@@ -1,0 +1,157 @@
+"""Pins for the oracle's MXFP4 path and block Hadamard (CPU only).
+
+Sources: "Bridging the Gap Between Promise and Performance for Microscaling
+FP4 Quantization" (gist.science, arXiv 2509.23202), technical summary sec. 1
+(MXFP4: 32-element groups, power-of-two E8M0 scales) and sec. 2 (MSE-optimised
+grid; fused block Hadamard micro-rotation, orthogonal); TORQ summary (arXiv
+2605.19561) sec. 2.B (S-step maps the block maximum onto the largest code).
+The e0-1..e0+1 window itself has no optimality statement on the pages: beyond
+the defined computation it is parity unpinned.
+"""
+import numpy as np
+import pytest
+from scipy.linalg import hadamard
+
+import synth
+from fp64_check import block_losses, unpack_nibbles
+
+RTOL_SUM32 = 6e-6        # rounding of a 32-term binary32 sequential sum of squares
+
+
+def test_hadamard_scale_is_rn_inverse_sqrt32(orc):
+    c = np.float32(1.0 / np.sqrt(np.float64(32.0)))
+    assert np.float32(orc.hadamard_scale()) == c
+    assert np.float32(orc.hadamard_scale()).view(np.uint32) == 0x3E3504F3
+
+
+@pytest.mark.parametrize("j", [0, 1, 5, 16, 31])
+@pytest.mark.parametrize("mask", [0, 0xFFFFFFFF, 0xA5A5A5A5])
+def test_hadamard_basis_vectors_closed_form(orc, j, mask):
+    x = np.zeros(32, dtype=np.float32)
+    x[j] = 1.0
+    y = orc.hadamard32(x, mask)
+    c = np.float32(orc.hadamard_scale())
+    sigma = -1.0 if (mask >> j) & 1 else 1.0
+    want = np.array([sigma * (-1) ** bin(i & j).count("1") for i in range(32)], dtype=np.float32) * c
+    np.testing.assert_array_equal(y, want)
+
+
+def test_hadamard_matches_sylvester_matrix(orc):
+    rng = np.random.default_rng(3)
+    H = hadamard(32).astype(np.float64)          # natural (Sylvester) order
+    for _ in range(50):
+        x = (rng.standard_t(3, size=32) * 0.02).astype(np.float32)
+        mask = int(rng.integers(0, 2 ** 32))
+        sig = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(32)])
+        want = H @ (sig * x.astype(np.float64)) / np.sqrt(32.0)
+        got = orc.hadamard32(x, mask).astype(np.float64)
+        # 5 stages of rounded adds plus one rounded multiply
+        bound = 8 * 2.0 ** -24 * np.sqrt(32.0) * np.abs(x).max() * 6
+        assert np.max(np.abs(got - want)) <= bound
+
+
+def test_hadamard_is_orthogonal(orc):
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal(32).astype(np.float32)
+    y = orc.hadamard32(x, 0)
+    z = orc.hadamard32(y, 0)
+    np.testing.assert_allclose(z, x, rtol=0, atol=1e-5 * np.abs(x).max())
+    assert abs(np.sum(y.astype(np.float64) ** 2) / np.sum(x.astype(np.float64) ** 2) - 1) < 1e-6
+
+
+@pytest.mark.parametrize("amax,e0", [(0.0, -127), (6.0, 0), (6.0000005, 1), (3.0, -1), (4.0, 0),
+                                     (1.5, -2), (1.5000001, -1), (2.0 ** -130, -127),
+                                     (3.0e38, 126)])
+def test_centre_exponent_cases(orc, amax, e0):
+    assert orc.mx_centre_exponent(amax) == e0
+
+
+def test_centre_exponent_property(orc):
+    rng = np.random.default_rng(5)
+    a = np.exp2(rng.uniform(-120, 120, size=20000)).astype(np.float32)
+    for v in a:
+        e = orc.mx_centre_exponent(v)
+        assert 6.0 * 2.0 ** e >= v and 6.0 * 2.0 ** (e - 1) < v
+
+
+def test_grid_exact_blocks(orc):
+    rng = np.random.default_rng(6)
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6], dtype=np.float64)
+    rows = []
+    ks = [-10, -3, 0, 4]
+    for k in ks:
+        g = grid[rng.integers(0, 8, size=32)] * np.where(rng.random(32) < 0.5, -1, 1)
+        g[3] = 6.0
+        rows.append(g * 2.0 ** k)
+    x = np.array(rows, dtype=np.float32).reshape(len(ks), 32)
+    out = orc.mxfp4_quant(x)
+    assert out["status"] == 0
+    np.testing.assert_array_equal(out["scales"].reshape(-1), np.array(ks) + 127)
+    np.testing.assert_array_equal(out["loss"], 0.0)
+    np.testing.assert_array_equal(out["y"], x)
+
+
+def _check_mx_against_fp64(v, out):
+    vb = v.reshape(-1, 32)
+    amax = np.abs(vb).max(axis=1)
+    import oracle
+    e0 = np.array([oracle.mx_centre_exponent(a) for a in amax])
+    cand = np.clip(e0[:, None] + np.arange(-1, 2), -127, 127)
+    d = np.exp2(cand.astype(np.float64)).astype(np.float32)
+    inv = np.exp2(-cand.astype(np.float64)).astype(np.float32)
+    loss64, codes, y32 = block_losses(vb, d, inv)
+    chosen = out["scales"].reshape(-1).astype(np.int64) - 127
+    k = np.argmax(cand == chosen[:, None], axis=1)
+    assert np.all(cand[np.arange(len(k)), k] == chosen)
+    picked = loss64[np.arange(len(k)), k]
+    assert np.all(picked <= loss64.min(axis=1) * (1 + 2 * RTOL_SUM32) + 1e-37)
+    np.testing.assert_allclose(out["loss"].reshape(-1), picked, rtol=RTOL_SUM32, atol=1e-37)
+    np.testing.assert_array_equal(unpack_nibbles(out["codes"]).reshape(-1, 32), codes[np.arange(len(k)), k])
+    np.testing.assert_array_equal(out["y"].reshape(-1, 32), y32[np.arange(len(k)), k])
+
+
+def test_mxfp4_plain_against_fp64(orc):
+    x = synth.t_weight(64, 512, nu=3, scale=0.015, seed=21).float().numpy()
+    out = orc.mxfp4_quant(x)
+    assert out["status"] == 0
+    np.testing.assert_array_equal(out["rotated"], x)
+    _check_mx_against_fp64(x, out)
+
+
+def test_mxfp4_hadamard_against_fp64(orc):
+    x = synth.t_weight(64, 512, nu=3, scale=0.015, seed=22).float().numpy()
+    masks = synth.sign_masks(512, seed=22)
+    out = orc.mxfp4_quant(x, sign_masks=masks)
+    assert out["status"] == 0
+    rot = np.stack([np.concatenate([orc.hadamard32(x[r, 32 * g:32 * g + 32], masks[g])
+                                    for g in range(16)]) for r in range(64)])
+    np.testing.assert_array_equal(out["rotated"], rot)
+    _check_mx_against_fp64(rot, out)
+
+
+def test_mxfp4_sweep_not_worse_than_centre(orc):
+    """Loss at the chosen exponent never exceeds the loss at e0 (fp64 check)."""
+    x = synth.t_weight(32, 1024, nu=3, scale=0.015, seed=23).float().numpy()
+    out = orc.mxfp4_quant(x)
+    xb = x.reshape(-1, 32)
+    import oracle
+    e0 = np.array([oracle.mx_centre_exponent(a) for a in np.abs(xb).max(axis=1)])
+    d = np.exp2(e0.astype(np.float64)).astype(np.float32)[:, None]
+    inv = np.exp2(-e0.astype(np.float64)).astype(np.float32)[:, None]
+    l0, _, _ = block_losses(xb, d, inv)
+    assert np.all(out["loss"].reshape(-1) <= l0[:, 0] * (1 + 2 * RTOL_SUM32))
+
+
+def test_mxfp4_nonfinite_status(orc):
+    x = np.ones((2, 64), dtype=np.float32)
+    x[1, 40] = np.inf
+    assert orc.mxfp4_quant(x)["status"] == orc.STATUS_NONFINITE
+    x[1, 40] = np.nan
+    assert orc.mxfp4_quant(x)["status"] == orc.STATUS_NONFINITE
+
+
+def test_mxfp4_dequant_reproduces_reconstruction(orc):
+    x = synth.t_weight(16, 256, nu=3, scale=0.015, seed=24).float().numpy()
+    out = orc.mxfp4_quant(x, sign_masks=synth.sign_masks(256, seed=1))
+    y = orc.mxfp4_dequant(out["codes"], out["scales"], 16, 256)
+    np.testing.assert_array_equal(y, out["y"])
