@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Throughput of the FP4 weight quantizer on a Llama-3-8B-shaped model.
+
+Workload (one "step"): every linear weight of a synthetic Llama-3-8B-shaped
+model -- 32 layers x {q, o: 4096x4096; k, v: 1024x4096; gate, up: 14336x4096;
+down: 4096x14336}, 224 bf16 tensors, 6.98e9 elements, Student-t(4) * 0.02 --
+is quantized to NVFP4 (global absmax, then the ScaleSweep MSE window search)
+and to MXFP4 (E8M0 exponent sweep); both emit packed codes, scales and the bf16
+reconstruction.  Inputs (13.96 GB) are resident in HBM and larger than L2, so
+no L2 flush is needed between steps.  The step is captured once as a CUDA graph
+and replayed.
+
+Metric: weight GB/s of bf16 input quantized (2 bytes x elements / time), whole
+job over all ranks; also elements/s and the fraction of the HBM roofline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun each rank quantizes its own copy of the model (seeded by rank):
+weak scaling, no collective on the data path; ranks synchronise only around
+the timed region and the slowest rank's time is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+
+METRIC = "weight GB/s (bf16 in) quantized to NVFP4/MXFP4 at 1 B200; % of HBM roofline"
+WORKLOAD = "llama3-8b-shaped whole-model pass: 224 bf16 linear weights -> NVFP4-MSE + MXFP4"
+# algorithmic bytes per element (bf16 in): absmax read 2; NVFP4 sweep read 2 + codes 0.5 +
+# scales 1/16 + bf16 deq 2; MXFP4 read 2 + codes 0.5 + scales 1/32 + bf16 deq 2
+B_ABSMAX = 2.0
+B_NVFP4 = 2.0 + 0.5 + 1.0 / 16 + 2.0
+B_MXFP4 = 2.0 + 0.5 + 1.0 / 32 + 2.0
+# fp32 operations the definition needs per element and candidate:
+# r = x*inv, E2M1(r), y = q*d, e = x - y, e*e, L + e*e
+OPS_PER_ELEM_CAND = 6
+NVFP4_MSE_CANDIDATES = 11
+SM_FP32_LANES = 128
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", 6650.0)), "measured", float(d.get("sm_max_mhz", 1965.0))
+    return 6650.0, "fallback", 1965.0
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except Exception as e:     # no nvidia-smi: report that instead of clocks
+            log("clock sampling unavailable:", e)
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- workload
+
+class Model:
+    """Device buffers of the whole-model pass and the launch sequence of one step."""
+
+    def __init__(self, fq, dev, seed: int, with_events: bool):
+        import synth
+        self.fq = fq
+        self.dev = dev
+        self.shapes = synth.llama3_8b_shapes()
+        self.w, self.out = [], []
+        t0 = time.time()
+        for i, (name, r, c) in enumerate(self.shapes):
+            self.w.append(synth.llama3_8b_tensor(i, r, c, seed=seed, device=dev))
+            kw = dict(device=dev)
+            self.out.append(dict(
+                amax=torch.empty(1, dtype=torch.float32, **kw),
+                S=torch.empty(1, dtype=torch.float32, **kw),
+                nv_codes=torch.empty((r, c // 2), dtype=torch.uint8, **kw),
+                nv_scales=torch.empty((r, c // 16), dtype=torch.uint8, **kw),
+                nv_deq=torch.empty((r, c), dtype=torch.bfloat16, **kw),
+                mx_codes=torch.empty((r, c // 2), dtype=torch.uint8, **kw),
+                mx_scales=torch.empty((r, c // 32), dtype=torch.uint8, **kw),
+                mx_deq=torch.empty((r, c), dtype=torch.bfloat16, **kw),
+            ))
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        torch.cuda.synchronize()
+        log(f"generated {len(self.w)} tensors in {time.time() - t0:.1f}s")
+        self.elements = sum(r * c for _, r, c in self.shapes)
+        self.events = None
+        if with_events:
+            self.events = [(torch.cuda.Event(enable_timing=True, external=True),
+                            torch.cuda.Event(enable_timing=True, external=True)) for _ in self.shapes]
+        self.launches_per_step = 3 * len(self.shapes)
+
+    def step(self, stream):
+        fq = self.fq
+        for i, (w, o) in enumerate(zip(self.w, self.out)):
+            fq.fp4q_global_absmax(w, o["amax"], stream)
+            if self.events is not None:
+                self.events[i][0].record(stream)
+            fq.fp4q_nvfp4_sweepmse(w, o["amax"], o["nv_codes"], o["nv_scales"], o["S"], o["nv_deq"],
+                                   None, self.status, stream)
+            if self.events is not None:
+                self.events[i][1].record(stream)
+            fq.fp4q_mxfp4_quant(w, o["mx_codes"], o["mx_scales"], o["mx_deq"], None, self.status, stream)
+
+    def sweep_ms(self):
+        return [a.elapsed_time(b) for a, b in self.events]
+
+
+def e2e_run(fq, model, steps, dev):
+    """Same step through the public API with host buffers: every step copies each bf16
+    weight from pinned host memory to the device, quantizes it, and copies the packed
+    result (NVFP4 codes + scales + S, MXFP4 codes + scales) back to pinned host memory.
+    Copies run on a copy stream and overlap the quantization of other tensors."""
+    host_w = [w.cpu().pin_memory() for w in model.w]
+    host_out = [dict(nv_codes=torch.empty_like(o["nv_codes"], device="cpu").pin_memory(),
+                     nv_scales=torch.empty_like(o["nv_scales"], device="cpu").pin_memory(),
+                     S=torch.empty(1, dtype=torch.float32).pin_memory(),
+                     mx_codes=torch.empty_like(o["mx_codes"], device="cpu").pin_memory(),
+                     mx_scales=torch.empty_like(o["mx_scales"], device="cpu").pin_memory())
+                for o in model.out]
+    h2d_bytes = sum(w.numel() * 2 for w in host_w)
+    d2h_bytes = sum(sum(t.numel() * t.element_size() for t in h.values()) for h in host_out)
+    compute = torch.cuda.Stream(device=dev)
+    h2d = torch.cuda.Stream(device=dev)
+    d2h = torch.cuda.Stream(device=dev)
+
+    def one_step():
+        for i, (hw, o, ho) in enumerate(zip(host_w, model.out, host_out)):
+            with torch.cuda.stream(h2d):
+                model.w[i].copy_(hw, non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(h2d)
+            compute.wait_event(ready)
+            fq.fp4q_global_absmax(model.w[i], o["amax"], compute)
+            fq.fp4q_nvfp4_sweepmse(model.w[i], o["amax"], o["nv_codes"], o["nv_scales"], o["S"],
+                                   o["nv_deq"], None, model.status, compute)
+            fq.fp4q_mxfp4_quant(model.w[i], o["mx_codes"], o["mx_scales"], o["mx_deq"], None,
+                                model.status, compute)
+            done = torch.cuda.Event()
+            done.record(compute)
+            d2h.wait_event(done)
+            with torch.cuda.stream(d2h):
+                for k in ho:
+                    ho[k].copy_(o[k], non_blocking=True)
+        torch.cuda.synchronize()
+
+    one_step()   # warm-up (also pages in the pinned buffers)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        one_step()
+    dt = (time.perf_counter() - t0) / steps
+    del host_w, host_out
+    return dt, h2d_bytes, d2h_bytes
+
+
+# --------------------------------------------------------------------------- CPU baseline
+
+def cpu_sample_rows():
+    return 256
+
+
+def cpu_baseline(seconds_hint=20.0):
+    """The oracle, as it stands, on a bounded sample of the workload: the first 256
+    rows of each of the 7 tensor shapes of one layer, NVFP4-MSE (absmax + sweep) and
+    MXFP4, all host cores (OpenMP)."""
+    import oracle
+    import synth
+    oracle.build()
+    rows = cpu_sample_rows()
+    shapes = synth.llama3_8b_shapes()[:7]
+    xs = [synth.llama3_8b_tensor(i, rows, c, seed=7).float().numpy() for i, (_, _, c) in enumerate(shapes)]
+    n = sum(x.size for x in xs)
+    t0 = time.perf_counter()
+    for x in xs:
+        g = oracle.global_absmax(x)
+        oracle.nvfp4_quant(x, S=oracle.global_scale(g))
+        oracle.mxfp4_quant(x)
+    dt = time.perf_counter() - t0
+    return {"value": 2.0 * n / dt / 1e9, "unit": "GB/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"first {rows} rows of each of the 7 tensor shapes of one layer "
+                      f"({n} elements): absmax + NVFP4-MSE sweep + MXFP4, {dt:.2f}s",
+            "elements_per_s": n / dt}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle timed on the host cores, per step one bounded
+    sample of the workload (see cpu_baseline)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    import synth
+    oracle.build()
+    rows = 64
+    shapes = synth.llama3_8b_shapes()[:7]
+    xs = [synth.llama3_8b_tensor(i, rows, c, seed=7).float().numpy() for i, (_, _, c) in enumerate(shapes)]
+    n = sum(x.size for x in xs)
+
+    def step():
+        for x in xs:
+            oracle.nvfp4_quant(x, S=oracle.global_scale(oracle.global_absmax(x)))
+            oracle.mxfp4_quant(x)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = 2.0 * n / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "sample_rows_per_tensor": rows,
+                                            "elements_per_step": n},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.max_threads(),
+                             "kind": "oracle", "sample": f"first {rows} rows of the 7 tensor shapes of one layer"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- single-kernel mode
+
+SINGLE_PATHS = {
+    # name: (bytes per element, kernel description)
+    "absmax": (B_ABSMAX, "absmax_kernel"),
+    "nvfp4-mse": (B_NVFP4, "nvfp4_sweep_kernel MSE"),
+    "nvfp4-wmse": (B_NVFP4, "nvfp4_sweep_kernel WMSE"),
+    "mxfp4": (B_MXFP4, "mxfp4_kernel"),
+    "mxfp4-hadamard": (B_MXFP4, "mxfp4_kernel Hadamard"),
+    "dequant-nvfp4": (0.5 + 1.0 / 16 + 2.0, "dequant_kernel NVFP4"),
+}
+
+
+def run_single(args):
+    """Time one kernel on one synthetic bf16 weight (`--shape RxC`), `--steps` launches
+    after `--warmup`, each launch timed with CUDA events on its stream; between
+    launches a 512 MB buffer is rewritten so that no launch starts with its input in L2.
+    Prints one JSON line (not the benchmark line)."""
+    import fp4_post_weight_grid_b200 as fq
+    from fp4_post_weight_grid_b200 import build as fbuild
+    import synth
+    fbuild.build()
+    rows, cols = (int(v) for v in args.shape.lower().split("x"))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = synth.t_weight(rows, cols, nu=4, scale=0.02, seed=11, device=dev)
+    imp = synth.importance_diag_xtx(cols=cols, tokens=256, seed=11, device=dev)
+    masks = torch.from_numpy(synth.sign_masks(cols, seed=11).view(np.int32)).to(dev)
+    amax = torch.empty(1, dtype=torch.float32, device=dev)
+    S = torch.empty(1, dtype=torch.float32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    sc16 = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+    sc32 = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
+    deq = torch.empty_like(w)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    fq.fp4q_global_absmax(w, amax)
+    fq.fp4q_nvfp4_sweepmse(w, amax, codes, sc16, S, deq, None, st)
+    stream = torch.cuda.current_stream()
+
+    def launch():
+        if args.single == "absmax":
+            fq.fp4q_global_absmax(w, amax, stream)
+        elif args.single == "nvfp4-mse":
+            fq.fp4q_nvfp4_sweepmse(w, amax, codes, sc16, S, deq, None, st, stream)
+        elif args.single == "nvfp4-wmse":
+            fq.fp4q_nvfp4_sweepwmse(w, amax, imp, codes, sc16, S, deq, None, st, stream)
+        elif args.single == "mxfp4":
+            fq.fp4q_mxfp4_quant(w, codes, sc32, deq, None, st, stream)
+        elif args.single == "mxfp4-hadamard":
+            fq.fp4q_mxfp4_quant_hadamard(w, masks, codes, sc32, deq, None, st, stream)
+        elif args.single == "dequant-nvfp4":
+            fq.fp4q_dequant(fq.NVFP4, codes, sc16, S, rows, cols, deq, stream)
+
+    times = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xFF)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        launch()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(a.elapsed_time(b))
+    hbm_peak, peak_kind, _ = load_peaks()
+    per_elem, kname = SINGLE_PATHS[args.single]
+    n = rows * cols
+    med = statistics.median(times)
+    gbs = per_elem * n / (med * 1e-3) / 1e9
+    print(json.dumps({"single": args.single, "kernel": kname, "shape": [rows, cols],
+                      "ms_median": med, "ms_min": min(times), "input_gbs": 2.0 * n / (med * 1e-3) / 1e9,
+                      "algorithmic_gbs": gbs, "hbm_peak": hbm_peak, "peak_kind": peak_kind,
+                      "hbm_frac": gbs / hbm_peak, "status": int(st.item())}), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--single", choices=sorted(SINGLE_PATHS), default=None,
+                    help="time one kernel on one tensor instead of the benchmark step")
+    ap.add_argument("--shape", default="16384x8192")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.single:
+        return run_single(args)
+
+    import fp4_post_weight_grid_b200 as fq
+    from fp4_post_weight_grid_b200 import build as fbuild
+    fbuild.build()
+    fq.load()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    model = Model(fq, dev, seed=5 + 1000 * rank, with_events=True)
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        model.step(stream)                       # eager warm-up before capture
+        stream.synchronize()
+        with torch.cuda.graph(graph, stream=stream):
+            model.step(stream)
+    for _ in range(max(args.warmup, 3) - 1):
+        graph.replay()
+    torch.cuda.synchronize()
+    if int(model.status.item()) != 0:
+        raise RuntimeError(f"device status {int(model.status.item())} during warm-up")
+
+    clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    clocks.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        t_end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    # the NVFP4 sweep kernel: per-launch durations of the last timed step
+    sweep_ms = model.sweep_ms()
+    status = int(model.status.item())
+
+    hbm_peak, peak_kind, sm_max = load_peaks()
+    n = model.elements
+    bytes_in = 2.0 * n * world
+    value = bytes_in / (ms * 1e-3) / 1e9
+    sweep_total_ms = sum(sweep_ms)
+    sweep_bytes = B_NVFP4 * n
+    sweep_gbs = sweep_bytes / (sweep_total_ms * 1e-3) / 1e9
+    clock_mhz = clk.get("sm_mhz") or sm_max
+    alu_peak = 148 * SM_FP32_LANES * clock_mhz * 1e6 / 1e12          # Tlane-op/s
+    alu_achieved = OPS_PER_ELEM_CAND * NVFP4_MSE_CANDIDATES * n / (sweep_total_ms * 1e-3) / 1e12
+    hbm_frac = sweep_gbs / hbm_peak
+    alu_frac = alu_achieved / alu_peak
+    if alu_frac > hbm_frac:
+        roof = {"bound": "alu", "achieved": alu_achieved, "peak": alu_peak, "unit": "Tlane-op/s",
+                "frac": alu_frac, "traffic": None, "kernel": "nvfp4_sweep_kernel (MSE, bf16)",
+                "peak_basis": f"148 SMs x 128 fp32 lanes x {clock_mhz:.0f} MHz median SM clock",
+                "hbm": {"achieved": sweep_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_frac,
+                        "peak_kind": peak_kind}}
+    else:
+        roof = {"bound": "hbm", "achieved": sweep_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_frac,
+                "traffic": None, "kernel": "nvfp4_sweep_kernel (MSE, bf16)", "peak_kind": peak_kind}
+    step_bytes = (B_ABSMAX + B_NVFP4 + B_MXFP4) * n
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tensors": len(model.shapes), "elements": n,
+                   "input_bytes": 2 * n, "l2": "inputs 13.96 GB > 126 MB L2, no flush",
+                   "parallelism": f"replicas x{world} (weak)", "graph": "one CUDA graph per step"},
+        "elements_per_s": n * world / (ms * 1e-3),
+        "hbm_frac_step": step_bytes / (ms * 1e-3) / 1e9 / hbm_peak,
+        "roofline": roof,
+        "gpu_launches": model.launches_per_step * args.steps,
+        "clocks": clk,
+        "status": status,
+    }
+    if rank == 0:
+        try:
+            e2e_dt, h2d, d2h = e2e_run(fq, model, max(1, args.e2e_steps), dev)
+            line["e2e"] = {"value": 2.0 * n / e2e_dt / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_dt * 1e3}
+        except Exception as e:   # report, do not hide
+            line["e2e"] = {"value": None, "unit": "GB/s", "error": repr(e)}
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        del graph
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

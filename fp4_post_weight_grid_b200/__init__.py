@@ -1,0 +1,314 @@
+"""Python binding of libfp4q, the sm_100a block-scaled FP4 weight quantizer.
+
+Argument marshalling only: every step of the quantization runs in the CUDA
+kernels behind the C ABI of ``include/fp4q.h``.  PyTorch supplies device
+memory and streams.  The functions named like the C entry points
+(``fp4q_global_absmax``, ``fp4q_nvfp4_sweepmse``, ``fp4q_nvfp4_sweepwmse``,
+``fp4q_mxfp4_quant``, ``fp4q_mxfp4_quant_hadamard``, ``fp4q_dequant``) take
+caller-allocated CUDA tensors, check their devices, dtypes and sizes, and
+enqueue the call on the current torch stream.  ``nvfp4_quantize``,
+``mxfp4_quantize`` and ``dequantize`` allocate the outputs with torch and call
+the same entry points.
+
+There is no CPU fallback: if ``libfp4q.so`` has not been built, or no CUDA
+device is visible, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import NamedTuple, Optional
+
+import torch
+
+__all__ = [
+    "Fp4qError", "library_path", "load", "version", "check_status",
+    "fp4q_global_absmax", "fp4q_nvfp4_sweepmse", "fp4q_nvfp4_sweepwmse", "fp4q_mxfp4_quant",
+    "fp4q_mxfp4_quant_hadamard", "fp4q_dequant", "fp4q_probe_e2m1", "fp4q_probe_e4m3",
+    "NVFP4Result", "MXFP4Result", "nvfp4_quantize", "mxfp4_quantize", "dequantize",
+    "FLAG_NONFINITE", "FLAG_RANGE",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libfp4q.so")
+_lib = None
+
+OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_NONFINITE, ERR_CUDA, ERR_RANGE = range(8)
+F32, BF16 = 0, 1
+NVFP4, MXFP4 = 0, 1
+FLAG_NONFINITE, FLAG_RANGE = 1, 2
+NVFP4_BLOCK, MXFP4_BLOCK = 16, 32
+EXPORTS = ("fp4q_version", "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_global_absmax",
+           "fp4q_nvfp4_sweepmse", "fp4q_nvfp4_sweepwmse", "fp4q_mxfp4_quant",
+           "fp4q_mxfp4_quant_hadamard", "fp4q_dequant", "fp4q_probe_e2m1", "fp4q_probe_e4m3")
+
+
+class Fp4qError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = load()
+        msg = lib.fp4q_status_string(status).decode()
+        if status == ERR_CUDA:
+            msg += ": " + lib.fp4q_last_cuda_error().decode()
+        super().__init__(f"{where}: {msg} (status {status})")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load libfp4q.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                           "`python -m fp4_post_weight_grid_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.fp4q_version.restype = I
+    lib.fp4q_version.argtypes = []
+    lib.fp4q_status_string.restype = ctypes.c_char_p
+    lib.fp4q_status_string.argtypes = [I]
+    lib.fp4q_last_cuda_error.restype = ctypes.c_char_p
+    lib.fp4q_last_cuda_error.argtypes = []
+    sigs = {
+        "fp4q_global_absmax": [P, I, I64, P, P],
+        "fp4q_nvfp4_sweepmse": [P, I, I64, I64, P, P, P, P, P, P, P, P],
+        "fp4q_nvfp4_sweepwmse": [P, I, I64, I64, P, P, P, P, P, P, P, P, P],
+        "fp4q_mxfp4_quant": [P, I, I64, I64, P, P, P, P, P, P],
+        "fp4q_mxfp4_quant_hadamard": [P, I, I64, I64, P, P, P, P, P, P, P],
+        "fp4q_dequant": [I, P, P, P, I64, I64, P, I, P],
+        "fp4q_probe_e2m1": [P, P, I64, P],
+        "fp4q_probe_e4m3": [P, P, I64, P],
+    }
+    for name, args in sigs.items():
+        fn = getattr(lib, name)
+        fn.restype = I
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def version() -> int:
+    return load().fp4q_version()
+
+
+# --------------------------------------------------------------------------- marshalling helpers
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def _dev(t: Optional[torch.Tensor], name: str, dtype=None, numel=None, device=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU fallback)")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {numel}")
+    return t.data_ptr() if t.numel() > 0 else None
+
+
+def _wdtype(w: torch.Tensor) -> int:
+    if w.dtype == torch.bfloat16:
+        return BF16
+    if w.dtype == torch.float32:
+        return F32
+    raise TypeError(f"weights must be bfloat16 or float32, got {w.dtype}")
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise Fp4qError(status, where)
+
+
+def _rc(w: torch.Tensor):
+    if w.dim() != 2:
+        raise ValueError("weights must be a 2-D [rows, cols] tensor")
+    return w.shape[0], w.shape[1]
+
+
+# --------------------------------------------------------------------------- C entry points
+
+def fp4q_global_absmax(x: torch.Tensor, d_amax: torch.Tensor, stream=None) -> None:
+    """d_amax[0] = max|x| (NaN if x holds a NaN).  ScaleSweep: S = max|x|/(256*6)."""
+    dev = x.device
+    xp = _dev(x, "x", device=dev)
+    ap = _dev(d_amax, "d_amax", torch.float32, 1, dev)
+    _check(load().fp4q_global_absmax(xp, _wdtype(x), x.numel(), ap, _stream(stream)),
+           "fp4q_global_absmax")
+
+
+def _nvfp4_args(w, d_amax, codes, scales, d_global_scale, deq, block_loss, d_status):
+    rows, cols = _rc(w)
+    dev = w.device
+    n = rows * cols
+    return (rows, cols, _dev(w, "w", device=dev), _dev(d_amax, "d_amax", torch.float32, 1, dev),
+            _dev(codes, "codes", torch.uint8, n // 2, dev),
+            _dev(scales, "scales", torch.uint8, n // NVFP4_BLOCK, dev),
+            _dev(d_global_scale, "d_global_scale", torch.float32, 1, dev),
+            _dev(deq, "deq", w.dtype, n, dev),
+            _dev(block_loss, "block_loss", torch.float32, n // NVFP4_BLOCK, dev),
+            _dev(d_status, "d_status", torch.int32, 1, dev))
+
+
+def fp4q_nvfp4_sweepmse(w, d_amax, codes, scales, d_global_scale, deq=None, block_loss=None,
+                        d_status=None, stream=None) -> None:
+    """NVFP4 ScaleSweep, MSE objective, window p-3..p+7 around s_base."""
+    rows, cols, wp, ap, cp, sp, gp, dp, lp, st = _nvfp4_args(w, d_amax, codes, scales,
+                                                            d_global_scale, deq, block_loss, d_status)
+    _check(load().fp4q_nvfp4_sweepmse(wp, _wdtype(w), rows, cols, ap, cp, sp, gp, dp, lp, st,
+                                      _stream(stream)), "fp4q_nvfp4_sweepmse")
+
+
+def fp4q_nvfp4_sweepwmse(w, d_amax, importance, codes, scales, d_global_scale, deq=None,
+                         block_loss=None, d_status=None, stream=None) -> None:
+    """NVFP4 ScaleSweep, importance-weighted MSE, window p-8..p+7."""
+    rows, cols, wp, ap, cp, sp, gp, dp, lp, st = _nvfp4_args(w, d_amax, codes, scales,
+                                                            d_global_scale, deq, block_loss, d_status)
+    ip = _dev(importance, "importance", torch.float32, cols, w.device)
+    _check(load().fp4q_nvfp4_sweepwmse(wp, _wdtype(w), rows, cols, ap, ip, cp, sp, gp, dp, lp, st,
+                                       _stream(stream)), "fp4q_nvfp4_sweepwmse")
+
+
+def _mx_args(w, codes, scales, deq, block_loss, d_status):
+    rows, cols = _rc(w)
+    dev = w.device
+    n = rows * cols
+    return (rows, cols, _dev(w, "w", device=dev), _dev(codes, "codes", torch.uint8, n // 2, dev),
+            _dev(scales, "scales", torch.uint8, n // MXFP4_BLOCK, dev),
+            _dev(deq, "deq", w.dtype, n, dev),
+            _dev(block_loss, "block_loss", torch.float32, n // MXFP4_BLOCK, dev),
+            _dev(d_status, "d_status", torch.int32, 1, dev))
+
+
+def fp4q_mxfp4_quant(w, codes, scales, deq=None, block_loss=None, d_status=None, stream=None) -> None:
+    """MXFP4, E8M0 exponent sweep e0-1..e0+1 per 32-element block."""
+    rows, cols, wp, cp, sp, dp, lp, st = _mx_args(w, codes, scales, deq, block_loss, d_status)
+    _check(load().fp4q_mxfp4_quant(wp, _wdtype(w), rows, cols, cp, sp, dp, lp, st, _stream(stream)),
+           "fp4q_mxfp4_quant")
+
+
+def fp4q_mxfp4_quant_hadamard(w, sign_masks, codes, scales, deq=None, block_loss=None,
+                              d_status=None, stream=None) -> None:
+    """MXFP4 after the fused random-sign 32-point block Hadamard rotation."""
+    rows, cols, wp, cp, sp, dp, lp, st = _mx_args(w, codes, scales, deq, block_loss, d_status)
+    mp = _dev(sign_masks, "sign_masks", (torch.int32, torch.uint32), cols // MXFP4_BLOCK, w.device)
+    _check(load().fp4q_mxfp4_quant_hadamard(wp, _wdtype(w), rows, cols, mp, cp, sp, dp, lp, st,
+                                            _stream(stream)), "fp4q_mxfp4_quant_hadamard")
+
+
+def fp4q_dequant(fmt: int, codes, scales, d_global_scale, rows: int, cols: int, out,
+                 stream=None) -> None:
+    """Decode codes + scales (+ S for NVFP4) into `out` (bf16 or fp32)."""
+    dev = out.device
+    bs = MXFP4_BLOCK if fmt == MXFP4 else NVFP4_BLOCK
+    n = rows * cols
+    cp = _dev(codes, "codes", torch.uint8, n // 2, dev)
+    sp = _dev(scales, "scales", torch.uint8, n // bs, dev)
+    gp = _dev(d_global_scale, "d_global_scale", torch.float32, 1, dev) if fmt == NVFP4 else None
+    op = _dev(out, "out", None, n, dev)
+    _check(load().fp4q_dequant(int(fmt), cp, sp, gp, rows, cols, op, _wdtype(out), _stream(stream)),
+           "fp4q_dequant")
+
+
+def fp4q_probe_e2m1(r: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    dev = r.device
+    _check(load().fp4q_probe_e2m1(_dev(r, "r", torch.float32, device=dev),
+                                  _dev(out, "out", torch.uint8, r.numel(), dev), r.numel(),
+                                  _stream(stream)), "fp4q_probe_e2m1")
+
+
+def fp4q_probe_e4m3(v: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    dev = v.device
+    _check(load().fp4q_probe_e4m3(_dev(v, "v", torch.float32, device=dev),
+                                  _dev(out, "out", torch.uint8, v.numel(), dev), v.numel(),
+                                  _stream(stream)), "fp4q_probe_e4m3")
+
+
+# --------------------------------------------------------------------------- allocating helpers
+
+class NVFP4Result(NamedTuple):
+    codes: torch.Tensor           # uint8 [rows, cols/2]
+    scales: torch.Tensor          # uint8 [rows, cols/16], E4M3 patterns
+    global_scale: torch.Tensor    # float32 [1], S
+    deq: Optional[torch.Tensor]   # input dtype [rows, cols]
+    block_loss: Optional[torch.Tensor]  # float32 [rows, cols/16]
+    amax: torch.Tensor            # float32 [1], max|w|
+    status: torch.Tensor          # int32 [1], FLAG_* bits
+
+
+class MXFP4Result(NamedTuple):
+    codes: torch.Tensor           # uint8 [rows, cols/2]
+    scales: torch.Tensor          # uint8 [rows, cols/32], E8M0 bytes
+    deq: Optional[torch.Tensor]
+    block_loss: Optional[torch.Tensor]
+    status: torch.Tensor
+
+
+def nvfp4_quantize(w: torch.Tensor, importance: Optional[torch.Tensor] = None, with_deq=True,
+                   with_loss=True, stream=None) -> NVFP4Result:
+    """Global absmax then the ScaleSweep (MSE, or WMSE when `importance` is given)."""
+    rows, cols = _rc(w)
+    dev = w.device
+    kw = dict(device=dev)
+    amax = torch.empty(1, dtype=torch.float32, **kw)
+    S = torch.empty(1, dtype=torch.float32, **kw)
+    status = torch.zeros(1, dtype=torch.int32, **kw)
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, **kw)
+    scales = torch.empty((rows, cols // NVFP4_BLOCK), dtype=torch.uint8, **kw)
+    deq = torch.empty_like(w) if with_deq else None
+    loss = torch.empty((rows, cols // NVFP4_BLOCK), dtype=torch.float32, **kw) if with_loss else None
+    fp4q_global_absmax(w, amax, stream)
+    if importance is None:
+        fp4q_nvfp4_sweepmse(w, amax, codes, scales, S, deq, loss, status, stream)
+    else:
+        fp4q_nvfp4_sweepwmse(w, amax, importance, codes, scales, S, deq, loss, status, stream)
+    return NVFP4Result(codes, scales, S, deq, loss, amax, status)
+
+
+def mxfp4_quantize(w: torch.Tensor, sign_masks: Optional[torch.Tensor] = None, with_deq=True,
+                   with_loss=True, stream=None) -> MXFP4Result:
+    """MXFP4 E8M0 sweep; block Hadamard first when `sign_masks` is given."""
+    rows, cols = _rc(w)
+    dev = w.device
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, cols // MXFP4_BLOCK), dtype=torch.uint8, device=dev)
+    deq = torch.empty_like(w) if with_deq else None
+    loss = torch.empty((rows, cols // MXFP4_BLOCK), dtype=torch.float32, device=dev) if with_loss else None
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    if sign_masks is None:
+        fp4q_mxfp4_quant(w, codes, scales, deq, loss, status, stream)
+    else:
+        fp4q_mxfp4_quant_hadamard(w, sign_masks, codes, scales, deq, loss, status, stream)
+    return MXFP4Result(codes, scales, deq, loss, status)
+
+
+def dequantize(fmt: int, codes: torch.Tensor, scales: torch.Tensor, global_scale=None,
+               dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+    rows, half = codes.shape
+    out = torch.empty((rows, half * 2), dtype=dtype, device=codes.device)
+    fp4q_dequant(fmt, codes, scales, global_scale, rows, half * 2, out, stream)
+    return out
+
+
+def check_status(status: torch.Tensor) -> int:
+    """Synchronize on the status word and raise on a device-reported flag."""
+    v = int(status.item())
+    if v & FLAG_NONFINITE:
+        raise Fp4qError(ERR_NONFINITE, "device status")
+    if v & FLAG_RANGE:
+        raise Fp4qError(ERR_RANGE, "device status")
+    return v

@@ -1,0 +1,208 @@
+// api.cu -- the C ABI declared in include/fp4q.h: argument checks, then one
+// stream-ordered launch per call.  No allocation, no host synchronization.
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "fp4q.h"
+#include "launch.h"
+
+namespace fp4q {
+
+int sm_count()
+{
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64 && cached[dev] > 0) return cached[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (dev < 64) cached[dev] = n;
+    return n;
+}
+
+}  // namespace fp4q
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "no error";
+
+fp4q_status after_launch()
+{
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) return FP4Q_OK;
+    std::strncpy(g_last_cuda_error, cudaGetErrorString(e), sizeof(g_last_cuda_error) - 1);
+    g_last_cuda_error[sizeof(g_last_cuda_error) - 1] = '\0';
+    return FP4Q_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool valid_dtype(fp4q_dtype dt) { return dt == FP4Q_F32 || dt == FP4Q_BF16; }
+
+// rows * cols without signed overflow
+bool shape_ok(int64_t rows, int64_t cols, int64_t block)
+{
+    if (rows < 0 || cols < 0 || cols % block != 0) return false;
+    if (cols != 0 && rows > INT64_MAX / 4 / cols) return false;
+    return true;
+}
+
+// FP4Q_OK with *empty set when there is nothing to do (the data pointers of an
+// empty tensor are not read and may be NULL).
+fp4q_status check_quant_args(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols, int64_t block,
+                             const void* codes, const void* scales, const int32_t* d_status,
+                             const void* deq, const float* loss, uintptr_t codes_align, bool* empty)
+{
+    *empty = false;
+    if (!valid_dtype(dt)) return FP4Q_ERR_DTYPE;
+    if (!shape_ok(rows, cols, block)) return FP4Q_ERR_SHAPE;
+    if (rows == 0 || cols == 0) { *empty = true; return FP4Q_OK; }
+    if (!w || !codes || !scales || !d_status) return FP4Q_ERR_NULL;
+    if (!aligned(w, 16) || !aligned(codes, codes_align) || (deq && !aligned(deq, 16)) ||
+        (loss && !aligned(loss, 4)) || !aligned(d_status, 4))
+        return FP4Q_ERR_ALIGN;
+    return FP4Q_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp4q_version(void) { return 10000; }
+
+const char* fp4q_status_string(fp4q_status status)
+{
+    switch (status) {
+    case FP4Q_OK: return "ok";
+    case FP4Q_ERR_NULL: return "a required pointer is NULL";
+    case FP4Q_ERR_SHAPE: return "invalid shape (negative size or cols not a multiple of the block size)";
+    case FP4Q_ERR_DTYPE: return "unknown dtype or format";
+    case FP4Q_ERR_ALIGN: return "pointer not aligned as required";
+    case FP4Q_ERR_NONFINITE: return "non-finite input";
+    case FP4Q_ERR_CUDA: return "CUDA launch error";
+    case FP4Q_ERR_RANGE: return "max|x| outside the supported range";
+    }
+    return "unknown status";
+}
+
+const char* fp4q_last_cuda_error(void) { return g_last_cuda_error; }
+
+fp4q_status fp4q_global_absmax(const void* x, fp4q_dtype dt, int64_t n, float* d_amax,
+                               fp4q_stream_t stream)
+{
+    if (!valid_dtype(dt)) return FP4Q_ERR_DTYPE;
+    if (n < 0) return FP4Q_ERR_SHAPE;
+    if (!d_amax || (n > 0 && !x)) return FP4Q_ERR_NULL;
+    if ((x && !aligned(x, 16)) || !aligned(d_amax, 4)) return FP4Q_ERR_ALIGN;
+    fp4q::launch_absmax(x, dt == FP4Q_BF16, n, d_amax, reinterpret_cast<cudaStream_t>(stream));
+    return after_launch();
+}
+
+static fp4q_status nvfp4_common(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                const float* d_amax, const float* importance, bool weighted,
+                                uint8_t* codes, uint8_t* scales, float* d_S, void* deq,
+                                float* loss, int32_t* d_status, fp4q_stream_t stream)
+{
+    bool empty = false;
+    fp4q_status st = check_quant_args(w, dt, rows, cols, FP4Q_NVFP4_BLOCK, codes, scales, d_status,
+                                      deq, loss, 8, &empty);
+    if (st != FP4Q_OK || empty) return st;
+    if (!d_amax || !d_S || (weighted && !importance)) return FP4Q_ERR_NULL;
+    if (!aligned(d_amax, 4) || !aligned(d_S, 4) || (weighted && !aligned(importance, 16)))
+        return FP4Q_ERR_ALIGN;
+    fp4q::launch_nvfp4_sweep(w, dt == FP4Q_BF16, rows, cols, d_amax, weighted ? importance : nullptr,
+                             codes, scales, d_S, deq, loss, d_status,
+                             reinterpret_cast<cudaStream_t>(stream));
+    return after_launch();
+}
+
+fp4q_status fp4q_nvfp4_sweepmse(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                const float* d_amax, uint8_t* codes, uint8_t* scales_e4m3,
+                                float* d_global_scale, void* deq, float* block_loss,
+                                int32_t* d_status, fp4q_stream_t stream)
+{
+    return nvfp4_common(w, dt, rows, cols, d_amax, nullptr, false, codes, scales_e4m3,
+                        d_global_scale, deq, block_loss, d_status, stream);
+}
+
+fp4q_status fp4q_nvfp4_sweepwmse(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                 const float* d_amax, const float* importance, uint8_t* codes,
+                                 uint8_t* scales_e4m3, float* d_global_scale, void* deq,
+                                 float* block_loss, int32_t* d_status, fp4q_stream_t stream)
+{
+    return nvfp4_common(w, dt, rows, cols, d_amax, importance, true, codes, scales_e4m3,
+                        d_global_scale, deq, block_loss, d_status, stream);
+}
+
+static fp4q_status mxfp4_common(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                const uint32_t* masks, bool rotate, uint8_t* codes, uint8_t* scales,
+                                void* deq, float* loss, int32_t* d_status, fp4q_stream_t stream)
+{
+    bool empty = false;
+    fp4q_status st = check_quant_args(w, dt, rows, cols, FP4Q_MXFP4_BLOCK, codes, scales, d_status,
+                                      deq, loss, 16, &empty);
+    if (st != FP4Q_OK || empty) return st;
+    if (rotate && !masks) return FP4Q_ERR_NULL;
+    if (rotate && !aligned(masks, 4)) return FP4Q_ERR_ALIGN;
+    fp4q::launch_mxfp4(w, dt == FP4Q_BF16, rows, cols, rotate ? masks : nullptr, codes, scales, deq,
+                       loss, d_status, reinterpret_cast<cudaStream_t>(stream));
+    return after_launch();
+}
+
+fp4q_status fp4q_mxfp4_quant(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                             uint8_t* codes, uint8_t* scales_e8m0, void* deq, float* block_loss,
+                             int32_t* d_status, fp4q_stream_t stream)
+{
+    return mxfp4_common(w, dt, rows, cols, nullptr, false, codes, scales_e8m0, deq, block_loss,
+                        d_status, stream);
+}
+
+fp4q_status fp4q_mxfp4_quant_hadamard(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                      const uint32_t* sign_masks, uint8_t* codes,
+                                      uint8_t* scales_e8m0, void* deq, float* block_loss,
+                                      int32_t* d_status, fp4q_stream_t stream)
+{
+    return mxfp4_common(w, dt, rows, cols, sign_masks, true, codes, scales_e8m0, deq, block_loss,
+                        d_status, stream);
+}
+
+fp4q_status fp4q_dequant(fp4q_format format, const uint8_t* codes, const uint8_t* scales,
+                         const float* d_global_scale, int64_t rows, int64_t cols, void* out,
+                         fp4q_dtype out_dt, fp4q_stream_t stream)
+{
+    if (format != FP4Q_NVFP4 && format != FP4Q_MXFP4) return FP4Q_ERR_DTYPE;
+    if (!valid_dtype(out_dt)) return FP4Q_ERR_DTYPE;
+    const bool mx = format == FP4Q_MXFP4;
+    if (!shape_ok(rows, cols, mx ? FP4Q_MXFP4_BLOCK : FP4Q_NVFP4_BLOCK)) return FP4Q_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return FP4Q_OK;
+    if (!codes || !scales || !out || (!mx && !d_global_scale)) return FP4Q_ERR_NULL;
+    if (!aligned(codes, mx ? 16 : 8) || !aligned(out, 16) || (!mx && !aligned(d_global_scale, 4)))
+        return FP4Q_ERR_ALIGN;
+    fp4q::launch_dequant(mx, codes, scales, d_global_scale, rows, cols, out, out_dt == FP4Q_BF16,
+                         reinterpret_cast<cudaStream_t>(stream));
+    return after_launch();
+}
+
+fp4q_status fp4q_probe_e2m1(const float* r, uint8_t* out, int64_t n, fp4q_stream_t stream)
+{
+    if (n < 0) return FP4Q_ERR_SHAPE;
+    if (n == 0) return FP4Q_OK;
+    if (!r || !out) return FP4Q_ERR_NULL;
+    if (!aligned(r, 4)) return FP4Q_ERR_ALIGN;
+    fp4q::launch_probe_e2m1(r, out, n, reinterpret_cast<cudaStream_t>(stream));
+    return after_launch();
+}
+
+fp4q_status fp4q_probe_e4m3(const float* v, uint8_t* out, int64_t n, fp4q_stream_t stream)
+{
+    if (n < 0) return FP4Q_ERR_SHAPE;
+    if (n == 0) return FP4Q_OK;
+    if (!v || !out) return FP4Q_ERR_NULL;
+    if (!aligned(v, 4)) return FP4Q_ERR_ALIGN;
+    fp4q::launch_probe_e4m3(v, out, n, reinterpret_cast<cudaStream_t>(stream));
+    return after_launch();
+}
+
+}  // extern "C"

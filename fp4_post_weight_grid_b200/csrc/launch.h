@@ -1,0 +1,32 @@
+// launch.h -- internal launchers behind the C ABI (include/fp4q.h).
+// Arguments are validated by api.cu before any of these is called.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp4q {
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+void launch_absmax(const void* x, bool bf16, int64_t n, float* d_amax, cudaStream_t s);
+
+// NVFP4 ScaleSweep: importance == nullptr selects MSE (window -3..+7), otherwise
+// WMSE (window -8..+7).
+void launch_nvfp4_sweep(const void* w, bool bf16, int64_t rows, int64_t cols, const float* d_amax,
+                        const float* importance, uint8_t* codes, uint8_t* scales, float* d_S,
+                        void* deq, float* loss, int32_t* d_status, cudaStream_t s);
+
+// MXFP4 with the E8M0 e0-1..e0+1 sweep; sign_masks != nullptr adds the block Hadamard.
+void launch_mxfp4(const void* w, bool bf16, int64_t rows, int64_t cols, const uint32_t* sign_masks,
+                  uint8_t* codes, uint8_t* scales, void* deq, float* loss, int32_t* d_status,
+                  cudaStream_t s);
+
+void launch_dequant(bool mx, const uint8_t* codes, const uint8_t* scales, const float* d_S,
+                    int64_t rows, int64_t cols, void* out, bool out_bf16, cudaStream_t s);
+
+void launch_probe_e2m1(const float* r, uint8_t* out, int64_t n, cudaStream_t s);
+void launch_probe_e4m3(const float* v, uint8_t* out, int64_t n, cudaStream_t s);
+
+}  // namespace fp4q

@@ -1,0 +1,226 @@
+/*
+ * fp4q.h -- C ABI of the block-scaled FP4 weight quantizer (CUDA, sm_100a).
+ *
+ * The library quantizes a dense row-major weight matrix W[rows][cols]
+ * (bf16 or fp32) to
+ *   NVFP4: 16-element blocks along a row, E2M1 elements, one E4M3 block scale
+ *          chosen by a ScaleSweep window search, one FP32 global scale S;
+ *   MXFP4: 32-element blocks along a row, E2M1 elements, one E8M0 block scale
+ *          chosen by an exponent sweep, optionally after a fused random-sign
+ *          32-point block Hadamard rotation.
+ * Sources: "Resumo Tecnico: ScaleSweep" (gist.science, arXiv 2606.07618),
+ * "Metodologia: ScaleSweep" secs. 1-3; "Bridging the Gap Between Promise and
+ * Performance for Microscaling FP4 Quantization" (gist.science, arXiv
+ * 2509.23202), technical summary secs. 1-3; "Resumo Tecnico: TORQ"
+ * (gist.science, arXiv 2605.19561) sec. 2.B.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.   Every pointer argument is DEVICE memory owned by the caller
+ *           (for example a torch tensor's data pointer) unless stated.  The
+ *           library allocates nothing and keeps no state between calls; it
+ *           may be called from several host threads at once.
+ * Streams.  Work is enqueued on `stream` (NULL = the legacy default stream)
+ *           and the call returns without waiting.  No call synchronizes,
+ *           allocates or copies through the host, so a sequence of calls can
+ *           be captured into a CUDA graph.
+ * Layout.   W is dense row-major, no leading-dimension stride.  Blocks never
+ *           cross a row (cols is a multiple of the block size), so block b of
+ *           the flattened tensor covers elements [b*B, b*B + B).
+ *           codes:  rows*cols/2 bytes; element 2j is the low nibble of byte j,
+ *                   element 2j+1 the high nibble; a nibble is sign<<3 | m
+ *                   with magnitude code m: 0:0 1:0.5 2:1 3:1.5 4:2 5:3 6:4 7:6.
+ *           scales: one byte per block, row-major [rows][cols/B]: an E4M3
+ *                   bit pattern 0x01..0x7E (NVFP4) or an E8M0 byte e+127
+ *                   (MXFP4).
+ *           deq:    the reconstruction q * d in the input dtype (RN to bf16).
+ *           block_loss: one fp32 per block, the selected candidate's loss.
+ * Errors.   Argument errors are returned at once and nothing is enqueued:
+ *           NULL required pointer (FP4Q_ERR_NULL), negative sizes or cols not
+ *           a multiple of the block size (FP4Q_ERR_SHAPE), unknown dtype or
+ *           format (FP4Q_ERR_DTYPE), a data pointer not aligned as stated
+ *           (FP4Q_ERR_ALIGN).  A failed launch returns FP4Q_ERR_CUDA (see
+ *           fp4q_last_cuda_error).  An empty tensor (rows or cols == 0) is
+ *           valid: after the dtype and shape checks the call returns FP4Q_OK,
+ *           enqueues nothing (except where stated) and reads none of its data
+ *           pointers, which may then be NULL.
+ *           Data-dependent errors are found on the device and OR-ed into the
+ *           caller's int32 status word *d_status as FP4Q_FLAG_* bits; the
+ *           caller zeroes it before the calls and reads it after a
+ *           synchronize.  When a flag is set the outputs are unspecified.
+ * Numerics. All arithmetic is IEEE binary32 with round-to-nearest-even, no
+ *           fused multiply-add and no flush-to-zero.  Each block's loss is
+ *           accumulated sequentially over its elements in column order:
+ *             r = x*inv; q = E2M1(r); y = q*d; e = x - y;
+ *             MSE: L = L + e*e        WMSE: L = L + w[col]*(e*e)
+ *           and candidates are visited in ascending order, the first one kept
+ *           and a later one taken only on a strictly smaller loss (ties go to
+ *           the smaller bit pattern).  E2M1 rounding is to nearest, ties to
+ *           the even code, saturating at 6; the sign of the input is kept,
+ *           so a negative value that rounds to zero encodes as 0x8.
+ */
+#ifndef FP4Q_H
+#define FP4Q_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* fp4q_stream_t;
+
+typedef enum {
+    FP4Q_OK = 0,
+    FP4Q_ERR_NULL = 1,
+    FP4Q_ERR_SHAPE = 2,
+    FP4Q_ERR_DTYPE = 3,
+    FP4Q_ERR_ALIGN = 4,
+    FP4Q_ERR_NONFINITE = 5,
+    FP4Q_ERR_CUDA = 6,
+    FP4Q_ERR_RANGE = 7
+} fp4q_status;
+
+typedef enum { FP4Q_F32 = 0, FP4Q_BF16 = 1 } fp4q_dtype;
+typedef enum { FP4Q_NVFP4 = 0, FP4Q_MXFP4 = 1 } fp4q_format;
+
+/* Bits OR-ed into *d_status by the device. */
+#define FP4Q_FLAG_NONFINITE 1  /* a NaN or Inf reached the scale search     */
+#define FP4Q_FLAG_RANGE     2  /* NVFP4: max|x| nonzero and outside [2^-64, 2^64] */
+
+#define FP4Q_NVFP4_BLOCK 16
+#define FP4Q_MXFP4_BLOCK 32
+
+/* Library version: major*10000 + minor*100 + patch. */
+int fp4q_version(void);
+
+/* Static description of a status code. */
+const char* fp4q_status_string(fp4q_status status);
+
+/* Text of the CUDA error behind the calling thread's last FP4Q_ERR_CUDA. */
+const char* fp4q_last_cuda_error(void);
+
+/*
+ * fp4q_global_absmax -- gmax = max |x_i| over n elements.
+ * ScaleSweep summary, "Metodologia" sec. 2: the FP32 global scale is
+ * S = max|x| / (256*6), so the whole tensor's max magnitude is needed first.
+ *   x       device, n elements of dtype `dt`, 16-byte aligned.
+ *   d_amax  device, one float; overwritten (the call first zeroes it, then
+ *           every thread block merges its maximum with an atomic max on the
+ *           bit pattern).  A NaN anywhere makes *d_amax a NaN; an Inf makes it
+ *           +Inf.  n == 0 leaves *d_amax = 0.
+ * Errors: FP4Q_ERR_NULL, FP4Q_ERR_SHAPE (n < 0), FP4Q_ERR_DTYPE,
+ * FP4Q_ERR_ALIGN, FP4Q_ERR_CUDA.
+ */
+fp4q_status fp4q_global_absmax(const void* x, fp4q_dtype dt, int64_t n, float* d_amax,
+                               fp4q_stream_t stream);
+
+/*
+ * fp4q_nvfp4_sweepmse -- NVFP4 ScaleSweep with the MSE objective.
+ * ScaleSweep summary, "Metodologia" secs. 1-3: S = gmax / 1536 (S = 1 when
+ * gmax == 0); per 16-element block s_base = E4M3_rne_sat(amax / (6*S)) (the
+ * block maximum relative to S rounded to FP8, pattern p); the candidates are
+ * the E4M3 patterns p-3 .. p+7 (Lemma 4.3 lower bound 4/5 s_base, Lemma 4.1
+ * upper bound 12/7 s_base) clipped to 0x01..0x7E; candidate p' has step
+ * d = E4M3(p')*S and reciprocal inv = 1/d; the block keeps the candidate with
+ * the smallest loss (conventions above).
+ *   w            device, rows*cols elements of `dt`, 16-byte aligned.
+ *   rows, cols   cols % 16 == 0.
+ *   d_amax       device, one float: max|w| from fp4q_global_absmax.
+ *   codes        device, rows*cols/2 bytes, 8-byte aligned.
+ *   scales_e4m3  device, rows*cols/16 bytes.
+ *   d_global_scale  device, one float: receives S.
+ *   deq          device or NULL, rows*cols elements of `dt`, 16-byte aligned.
+ *   block_loss   device or NULL, rows*cols/16 floats, 4-byte aligned.
+ *   d_status     device int32: FP4Q_FLAG_NONFINITE if gmax is NaN/Inf,
+ *                FP4Q_FLAG_RANGE if gmax is nonzero and outside [2^-64, 2^64].
+ */
+fp4q_status fp4q_nvfp4_sweepmse(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                const float* d_amax, uint8_t* codes, uint8_t* scales_e4m3,
+                                float* d_global_scale, void* deq, float* block_loss,
+                                int32_t* d_status, fp4q_stream_t stream);
+
+/*
+ * fp4q_nvfp4_sweepwmse -- NVFP4 ScaleSweep with the importance-weighted MSE.
+ * ScaleSweep summary, "Metodologia" sec. 1 (WMSE weights errors by importance
+ * scores from activation norms or Gram-matrix diagonals) and sec. 2 (the lower
+ * bound is set empirically to 1/2 s_base, offset -8): candidates p-8 .. p+7,
+ * loss L = L + importance[col]*(e*e).  Arguments as fp4q_nvfp4_sweepmse plus
+ *   importance   device, cols floats (one per input column), 16-byte aligned,
+ *                used as given (diag(X^T X) or any non-negative weights).
+ */
+fp4q_status fp4q_nvfp4_sweepwmse(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                 const float* d_amax, const float* importance, uint8_t* codes,
+                                 uint8_t* scales_e4m3, float* d_global_scale, void* deq,
+                                 float* block_loss, int32_t* d_status, fp4q_stream_t stream);
+
+/*
+ * fp4q_mxfp4_quant -- MXFP4 with an E8M0 exponent sweep.
+ * MR-GPTQ summary, technical sec. 1 (32-element groups, power-of-two E8M0
+ * scales) and sec. 2 (scales chosen to minimise the MSE); TORQ summary sec.
+ * 2.B (the block maximum maps onto the largest code).  Per 32-element block:
+ * e0 = the smallest e with 6*2^e >= amax (e0 = -127 for a zero block), clamped
+ * to [-127, 127]; the candidates e0-1, e0, e0+1 (clamped) use d = 2^e and
+ * inv = 2^-e with the MSE loss; the scale byte is e*+127.
+ *   w        device, rows*cols elements of `dt`, 16-byte aligned; cols % 32 == 0.
+ *   codes    device, rows*cols/2 bytes, 16-byte aligned.
+ *   scales_e8m0  device, rows*cols/32 bytes.
+ *   deq      device or NULL, rows*cols elements of `dt`, 16-byte aligned.
+ *   block_loss   device or NULL, rows*cols/32 floats.
+ *   d_status device int32: FP4Q_FLAG_NONFINITE if a block holds a NaN/Inf.
+ */
+fp4q_status fp4q_mxfp4_quant(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                             uint8_t* codes, uint8_t* scales_e8m0, void* deq, float* block_loss,
+                             int32_t* d_status, fp4q_stream_t stream);
+
+/*
+ * fp4q_mxfp4_quant_hadamard -- MXFP4 after a fused random-sign block Hadamard.
+ * MR-GPTQ summary, technical sec. 2 ("Rotacoes Online Fundidas": block
+ * Hadamard micro-rotations fused into the GPU kernels) and sec. 3.  Each
+ * 32-block is rotated in registers before the exponent sweep:
+ * y = c * H32 * diag(sigma) * x, sigma_j = -1 where bit j of
+ * sign_masks[col/32] is set, H32 the Sylvester (natural-order) Hadamard applied
+ * as five butterfly stages h = 1,2,4,8,16 ((a,b) -> (a+b, a-b)), then every
+ * element times c = RN(1/sqrt(32)).  The codes, scales, deq and loss are those
+ * of the rotated block (deq is in the rotated domain).
+ *   sign_masks  device, cols/32 uint32 (one mask per 32-column group, shared
+ *               by all rows), 4-byte aligned.
+ * Other arguments as fp4q_mxfp4_quant; FP4Q_FLAG_NONFINITE also covers a
+ * rotation that overflows.
+ */
+fp4q_status fp4q_mxfp4_quant_hadamard(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                      const uint32_t* sign_masks, uint8_t* codes,
+                                      uint8_t* scales_e8m0, void* deq, float* block_loss,
+                                      int32_t* d_status, fp4q_stream_t stream);
+
+/*
+ * fp4q_dequant -- decode codes and scales back to values.
+ * NVFP4: out = RN(q * RN(E4M3(s) * S)), S = *d_global_scale; MXFP4:
+ * out = q * 2^(b-127); then rounded to `out_dt`.  Reproduces the `deq` output
+ * of the quantizers bit for bit.  A NaN scale pattern (E4M3 0x7F/0xFF, E8M0
+ * 0xFF) decodes to NaN; E4M3 patterns with the sign bit decode as negative.
+ *   codes   device, rows*cols/2 bytes, 8-byte aligned (16 for MXFP4).
+ *   scales  device, rows*cols/16 (NVFP4) or rows*cols/32 (MXFP4) bytes.
+ *   d_global_scale  device float (NVFP4 only; ignored and may be NULL for MXFP4).
+ *   out     device, rows*cols elements of `out_dt`, 16-byte aligned.
+ */
+fp4q_status fp4q_dequant(fp4q_format format, const uint8_t* codes, const uint8_t* scales,
+                         const float* d_global_scale, int64_t rows, int64_t cols, void* out,
+                         fp4q_dtype out_dt, fp4q_stream_t stream);
+
+/*
+ * Diagnostic entry points: the device's element and scale rounding primitives
+ * applied to n floats, so that they can be compared with a reference codec.
+ *   fp4q_probe_e2m1: out[i] = E2M1 nibble of r[i] (sign<<3 | code).
+ *   fp4q_probe_e4m3: out[i] = E4M3 pattern of v[i] >= 0 (RNE, saturating).
+ * r/v device, 4-byte aligned; out device bytes.
+ */
+fp4q_status fp4q_probe_e2m1(const float* r, uint8_t* out, int64_t n, fp4q_stream_t stream);
+fp4q_status fp4q_probe_e4m3(const float* v, uint8_t* out, int64_t n, fp4q_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4Q_H */

@@ -1,0 +1,109 @@
+"""CPU checks of the C ABI library and the Python binding (no GPU needed).
+
+The library must load, export every entry point declared in include/fp4q.h,
+and the binding must refuse CPU tensors instead of falling back to the CPU.
+No compute call is made here.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def fq():
+    from fp4_post_weight_grid_b200 import build
+    build.build()
+    import fp4_post_weight_grid_b200 as m
+    m.load()
+    return m
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "fp4q.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp4q_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    names = _declared()
+    for want in ("fp4q_global_absmax", "fp4q_nvfp4_sweepmse", "fp4q_nvfp4_sweepwmse",
+                 "fp4q_mxfp4_quant", "fp4q_mxfp4_quant_hadamard", "fp4q_dequant"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(fq):
+    lib = ctypes.CDLL(fq.library_path())
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert sorted(fq.EXPORTS) == _declared()
+
+
+def test_version_and_status_strings(fq):
+    lib = fq.load()
+    assert lib.fp4q_version() >= 10000
+    for s in range(8):
+        assert lib.fp4q_status_string(s)
+    assert b"unknown" in lib.fp4q_status_string(99)
+
+
+def test_argument_errors_without_a_gpu(fq):
+    """Argument checks run before any CUDA call, so they work on a CPU-only host."""
+    lib = fq.load()
+    buf = ctypes.create_string_buffer(256)
+    p = ctypes.addressof(buf)
+    p16 = p + (-p % 16)
+    # bad dtype, bad shape, NULL pointers, misalignment
+    assert lib.fp4q_nvfp4_sweepmse(p16, 7, 1, 16, p16, p16, p16, p16, None, None, p16, None) == fq.ERR_DTYPE
+    assert lib.fp4q_nvfp4_sweepmse(p16, 1, 1, 17, p16, p16, p16, p16, None, None, p16, None) == fq.ERR_SHAPE
+    assert lib.fp4q_nvfp4_sweepmse(p16, 1, -1, 16, p16, p16, p16, p16, None, None, p16, None) == fq.ERR_SHAPE
+    assert lib.fp4q_nvfp4_sweepmse(None, 1, 1, 16, p16, p16, p16, p16, None, None, p16, None) == fq.ERR_NULL
+    assert lib.fp4q_nvfp4_sweepmse(p16 + 2, 1, 1, 16, p16, p16, p16, p16, None, None, p16, None) == fq.ERR_ALIGN
+    assert lib.fp4q_nvfp4_sweepwmse(p16, 1, 1, 16, p16, None, p16, p16, p16, None, None, p16, None) == fq.ERR_NULL
+    assert lib.fp4q_mxfp4_quant(p16, 1, 1, 48, p16, p16, None, None, p16, None) == fq.ERR_SHAPE
+    assert lib.fp4q_mxfp4_quant(p16, 1, 1, 32, p16 + 8, p16, None, None, p16, None) == fq.ERR_ALIGN
+    assert lib.fp4q_mxfp4_quant_hadamard(p16, 1, 1, 32, None, p16, p16, None, None, p16, None) == fq.ERR_NULL
+    assert lib.fp4q_dequant(5, p16, p16, p16, 1, 16, p16, 1, None) == fq.ERR_DTYPE
+    assert lib.fp4q_dequant(0, p16, p16, None, 1, 16, p16, 1, None) == fq.ERR_NULL
+    assert lib.fp4q_global_absmax(p16, 1, -5, p16, None) == fq.ERR_SHAPE
+    assert lib.fp4q_global_absmax(p16 + 4, 1, 5, p16, None) == fq.ERR_ALIGN
+    # empty tensors are valid and touch nothing
+    assert lib.fp4q_nvfp4_sweepmse(None, 1, 0, 16, None, None, None, None, None, None, None, None) == fq.OK
+    assert lib.fp4q_mxfp4_quant(None, 0, 5, 0, None, None, None, None, None, None) == fq.OK
+    assert lib.fp4q_dequant(1, None, None, None, 0, 32, None, 0, None) == fq.OK
+
+
+def test_binding_refuses_cpu_tensors(fq):
+    w = torch.zeros((4, 32), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        fq.fp4q_global_absmax(w, torch.zeros(1))
+    with pytest.raises(ValueError, match="CUDA"):
+        fq.nvfp4_quantize(w)
+
+
+def test_missing_library_fails_loudly(fq, monkeypatch, tmp_path):
+    monkeypatch.setattr(fq, "_lib", None)
+    monkeypatch.setattr(fq, "_LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        fq.load()
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "fp4_post_weight_grid_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in text.lower().replace("oracle-free", ""), f
+
+
+def test_oracle_and_library_share_no_source():
+    orc = open(os.path.join(ROOT, "oracle", "fp4q_oracle.c")).read()
+    assert "#include \"" not in orc          # the oracle includes only system headers
+    for f in os.listdir(os.path.join(ROOT, "fp4_post_weight_grid_b200", "csrc")):
+        assert "oracle" not in open(os.path.join(ROOT, "fp4_post_weight_grid_b200", "csrc", f)).read()
