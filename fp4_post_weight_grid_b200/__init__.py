@@ -134,9 +134,11 @@ def _check(status: int, where: str):
         raise Fp4qError(status, where)
 
 
-def _rc(w: torch.Tensor):
+def _rc(w: torch.Tensor, block: int = 1):
     if w.dim() != 2:
         raise ValueError("weights must be a 2-D [rows, cols] tensor")
+    if w.shape[1] % block:
+        raise Fp4qError(ERR_SHAPE, f"cols = {w.shape[1]} is not a multiple of the block size {block}")
     return w.shape[0], w.shape[1]
 
 
@@ -152,7 +154,7 @@ def fp4q_global_absmax(x: torch.Tensor, d_amax: torch.Tensor, stream=None) -> No
 
 
 def _nvfp4_args(w, d_amax, codes, scales, d_global_scale, deq, block_loss, d_status):
-    rows, cols = _rc(w)
+    rows, cols = _rc(w, NVFP4_BLOCK)
     dev = w.device
     n = rows * cols
     return (rows, cols, _dev(w, "w", device=dev), _dev(d_amax, "d_amax", torch.float32, 1, dev),
@@ -184,7 +186,7 @@ def fp4q_nvfp4_sweepwmse(w, d_amax, importance, codes, scales, d_global_scale, d
 
 
 def _mx_args(w, codes, scales, deq, block_loss, d_status):
-    rows, cols = _rc(w)
+    rows, cols = _rc(w, MXFP4_BLOCK)
     dev = w.device
     n = rows * cols
     return (rows, cols, _dev(w, "w", device=dev), _dev(codes, "codes", torch.uint8, n // 2, dev),
@@ -261,7 +263,7 @@ class MXFP4Result(NamedTuple):
 def nvfp4_quantize(w: torch.Tensor, importance: Optional[torch.Tensor] = None, with_deq=True,
                    with_loss=True, stream=None) -> NVFP4Result:
     """Global absmax then the ScaleSweep (MSE, or WMSE when `importance` is given)."""
-    rows, cols = _rc(w)
+    rows, cols = _rc(w, NVFP4_BLOCK)
     dev = w.device
     kw = dict(device=dev)
     amax = torch.empty(1, dtype=torch.float32, **kw)
@@ -282,7 +284,7 @@ def nvfp4_quantize(w: torch.Tensor, importance: Optional[torch.Tensor] = None, w
 def mxfp4_quantize(w: torch.Tensor, sign_masks: Optional[torch.Tensor] = None, with_deq=True,
                    with_loss=True, stream=None) -> MXFP4Result:
     """MXFP4 E8M0 sweep; block Hadamard first when `sign_masks` is given."""
-    rows, cols = _rc(w)
+    rows, cols = _rc(w, MXFP4_BLOCK)
     dev = w.device
     codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
     scales = torch.empty((rows, cols // MXFP4_BLOCK), dtype=torch.uint8, device=dev)

@@ -1,8 +1,9 @@
 """Build libfp4q.so in-tree with nvcc for sm_100a.
 
-Flags: -gencode arch=compute_100a,code=sm_100a -O3 -lineinfo and --fmad=false
-(no multiply-add contraction anywhere, so every binary32 operation is the
-separately rounded one the results are defined by).  ptxas resource usage of
+Flags: -gencode arch=compute_100a,code=sm_100a -O3 -lineinfo and --fmad=false,
+given to both the compiler and ptxas (no multiply-add contraction anywhere, so
+every binary32 operation is the separately rounded one the results are defined
+by).  ptxas resource usage of
 every kernel is written to _build/ptxas.log.
 """
 from __future__ import annotations
@@ -44,7 +45,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
     os.makedirs(os.path.join(HERE, "_build"), exist_ok=True)
-    cmd = [nvcc_path(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "--fmad=false",
+    cmd = [nvcc_path(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "--fmad=false", "-Xptxas", "--fmad=false",
            "-Xcompiler", "-fPIC", "-shared", "-Xptxas", "-v",
            "-I", os.path.join(ROOT, "include"),
            *[os.path.join(SRC, s) for s in SOURCES], "-o", LIB + ".tmp"]

@@ -47,6 +47,20 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b)
     return r;
 }
 
+// Product a*b of a pair, for a product that feeds an add or a subtract.
+// ptxas fuses a packed mul.rn.f32x2 followed by add/sub.rn.f32x2 into one
+// fused multiply-add even when contraction is disabled, which changes the
+// rounding.  Computing the product as fma(a, b, z) with z = (-0, -0) held in a
+// register gives exactly RN(a*b) (adding -0 changes no value, zero signs
+// included) and an fma result cannot be fused again.  `z` must come from a
+// runtime value (a kernel argument) so that it is not folded back into a mul.
+__device__ __forceinline__ uint64_t mul2_nofuse(uint64_t a, uint64_t b, uint64_t z)
+{
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(z));
+    return r;
+}
+
 // ---------------------------------------------------------------- E2M1
 // Two binary32 values -> one byte holding two E2M1 nibbles, `lo` in bits 0..3
 // and `hi` in bits 4..7 (the instruction stores its first source in the upper
@@ -88,6 +102,21 @@ __device__ __forceinline__ uint64_t e2m1x2_decode(uint32_t byte)
     float lo, hi;
     f16x2_to_f32(e2m1x2_to_f16x2(byte), lo, hi);
     return pk(lo, hi);
+}
+
+// Round a pair to E2M1 and return the rounded values as binary32, without
+// materialising the code byte (the byte stays in an 8-bit PTX register between
+// the two conversions).
+__device__ __forceinline__ uint64_t e2m1x2_round(float lo, float hi)
+{
+    uint32_t h2;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(h2) : "f"(hi), "f"(lo));
+    float a, b;
+    f16x2_to_f32(h2, a, b);
+    return pk(a, b);
 }
 
 // ---------------------------------------------------------------- E4M3

@@ -35,8 +35,9 @@ __global__ void __launch_bounds__(kThreads)
 mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
              const uint32_t* __restrict__ masks, uint8_t* __restrict__ codes,
              uint8_t* __restrict__ scales, T* __restrict__ deq, float* __restrict__ loss,
-             int32_t* __restrict__ d_status)
+             int32_t* __restrict__ d_status, float neg_zero)
 {
+    const uint64_t z2 = pk(neg_zero, neg_zero);
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     for (int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x; b < nblocks; b += stride) {
         float x[32];
@@ -85,9 +86,9 @@ mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
                 const uint64_t aa = pk(a, a);
                 float ra, rb;
                 upk(mul2(aa, inv2), ra, rb);
-                const uint64_t q2 = e2m1x2_decode(e2m1x2(ra, rb));
-                const uint64_t e2 = sub2(aa, mul2(q2, d2));
-                L2 = add2(L2, mul2(e2, e2));
+                const uint64_t q2 = e2m1x2_round(ra, rb);
+                const uint64_t e2 = sub2(aa, mul2_nofuse(q2, d2, z2));
+                L2 = add2(L2, mul2_nofuse(e2, e2, z2));
             }
             float La, Lb;
             upk(L2, La, Lb);
@@ -132,7 +133,7 @@ void launch_typed(const void* w, int64_t rows, int64_t cols, const uint32_t* mas
     if (grid < 1) grid = 1;
     mxfp4_kernel<T, HAD><<<(unsigned)grid, kThreads, 0, s>>>(
         static_cast<const T*>(w), nblocks, cols / 32, masks, codes, scales, static_cast<T*>(deq),
-        loss, d_status);
+        loss, d_status, -0.0f);
 }
 
 }  // namespace

@@ -21,7 +21,9 @@
 // inv_k+1) is one packed multiply, one cvt.e2m1x2 rounds both to E2M1 (ties to
 // even, saturating), one cvt back to f16x2 and two exact widenings give
 // (q_k, q_k+1); then y = q*d, e = |x| - y, e*e (and w*(e*e)) and L += are four
-// packed RN operations.  Working on |x| gives the same e*e as the signed value
+// packed RN operations (the two products that feed an add are issued as fma
+// with a -0 addend so that ptxas cannot fuse them into the add; see
+// mul2_nofuse).  Working on |x| gives the same e*e as the signed value
 // because round-to-nearest is symmetric.  Per-candidate steps d = RN(E4M3(p)*S)
 // and inv = RN(1/d) for all 126 patterns are computed once per thread block
 // into shared memory.  The window is clamped to 0x01..0x7E by clamping each
@@ -42,9 +44,10 @@ nvfp4_sweep_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_
                    const float* __restrict__ d_amax, const float* __restrict__ importance,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                    float* __restrict__ d_S, T* __restrict__ deq, float* __restrict__ loss,
-                   int32_t* __restrict__ d_status)
+                   int32_t* __restrict__ d_status, float neg_zero)
 {
     constexpr int NC = (NREAL + 1) & ~1;   // candidates evaluated in pairs
+    const uint64_t z2 = pk(neg_zero, neg_zero);
     __shared__ float2 step[128];           // (d, inv) per E4M3 pattern
 
     const float gmax = __ldg(d_amax);
@@ -106,10 +109,10 @@ nvfp4_sweep_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_
             for (int i = 0; i < 16; ++i) {
                 float ra, rb;
                 upk(mul2(aa[i], inv2), ra, rb);
-                const uint64_t q2 = e2m1x2_decode(e2m1x2(ra, rb));
-                const uint64_t e2 = sub2(aa[i], mul2(q2, d2));
-                uint64_t s2 = mul2(e2, e2);
-                if (WMSE) s2 = mul2(ww[i], s2);
+                const uint64_t q2 = e2m1x2_round(ra, rb);
+                const uint64_t e2 = sub2(aa[i], mul2_nofuse(q2, d2, z2));
+                uint64_t s2 = mul2_nofuse(e2, e2, z2);
+                if (WMSE) s2 = mul2_nofuse(ww[i], s2, z2);
                 L2 = add2(L2, s2);
             }
             float La, Lb;
@@ -157,7 +160,7 @@ void launch_typed(const void* w, int64_t rows, int64_t cols, const float* d_amax
     if (grid < 1) grid = 1;
     nvfp4_sweep_kernel<T, LO, NREAL, WMSE><<<(unsigned)grid, kThreads, 0, s>>>(
         static_cast<const T*>(w), nblocks, cols / 16, d_amax, importance, codes, scales, d_S,
-        static_cast<T*>(deq), loss, d_status);
+        static_cast<T*>(deq), loss, d_status, -0.0f);
 }
 
 }  // namespace
