@@ -22,6 +22,7 @@
 // memory budget of ~4.5 bytes per element.
 #include "device.cuh"
 #include "launch.h"
+#include "screen.cuh"
 
 namespace fp4q {
 
@@ -70,55 +71,101 @@ mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
             e0 = a - 2 + ((abits & 0x7FFFFFu) > 0x400000u ? 1 : 0);  // 6*2^(a-2) = 1.5*2^a
             e0 = min(max(e0, -127), 127);
         }
-        const int ea = max(e0 - 1, -127), ec = min(e0 + 1, 127);
-        float best = 0.0f;
-        int be = ea;
+        // candidate k = 0, 1, 2 is the exponent e0 - 1 + k, clamped to [-127, 127]
+#define FP4Q_EK(k) min(max(e0 - 1 + (k), -127), 127)
+
+        // 1. screen the three exponents in units of 2^e0 (S = 2^e0, v = 2^(e-e0))
+        const float inv0 = exp2i(-e0);
+        float alpha2 = 0.0f;
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const int e_lo = k == 0 ? ea : ec;
-            const int e_hi = k == 0 ? e0 : ec;
-            const uint64_t inv2 = pk(exp2i(-e_lo), exp2i(-e_hi));
-            const uint64_t d2 = pk(exp2i(e_lo), exp2i(e_hi));
+        for (int j = 0; j < 32; ++j) {
+            const float as = fabsf(x[j]) * inv0;
+            alpha2 = fmaf(as, as, alpha2);
+        }
+        alpha2 *= 1.0f + 0x1p-16f;
+        const float tS = 0x1p-70f * inv0;
+        const float tau = tS * tS + 0x1p-120f;
+        float lam[4];
+#pragma unroll
+        for (int k = 0; k < 4; k += 2) {
+            const int ea = FP4Q_EK(k), eb = FP4Q_EK(min(k + 1, 2));
+            const uint64_t inv2 = pk(exp2i(-ea), exp2i(-eb));
             uint64_t L2 = pk(0.0f, 0.0f);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const float a = fabsf(x[i]);
-                const uint64_t aa = pk(a, a);
                 float ra, rb;
-                upk(mul2(aa, inv2), ra, rb);
-                const uint64_t q2 = e2m1x2_round(ra, rb);
-                const uint64_t e2 = sub2(aa, mul2_nofuse(q2, d2, z2));
-                L2 = add2(L2, mul2_nofuse(e2, e2, z2));
+                upk(mul2(pk(a, a), inv2), ra, rb);
+                const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
+                L2 = fma2(et, et, L2);
             }
-            float La, Lb;
-            upk(L2, La, Lb);
-            if (k == 0 || La < best) { best = La; be = e_lo; }
-            if (Lb < best) { best = Lb; be = e_hi; }
+            upk(mul2(L2, pk(exp2i(2 * (ea - e0)), exp2i(2 * (eb - e0)))), lam[k], lam[k + 1]);
         }
+        const float M = fminf(fminf(lam[0], lam[1]), lam[2]);
+        const float T = survivor_threshold(M, alpha2, tau);
+        uint32_t mask = (lam[0] <= T ? 1u : 0u) | (lam[1] <= T ? 2u : 0u) | (lam[2] <= T ? 4u : 0u);
+        if (mask == 0) mask = 7u;                  // unreachable for finite inputs; evaluate all
+
+        // 2. verify: exact loss of the survivors, first minimum wins
+        int be;
+        if ((mask & (mask - 1)) == 0) {
+            be = FP4Q_EK(__ffs(mask) - 1);
+        } else {
+            float best = 0.0f;
+            bool first = true;
+            be = FP4Q_EK(0);
+            while (mask) {
+                const int k = __ffs(mask) - 1;
+                mask &= mask - 1;
+                const int e = FP4Q_EK(k);
+                const uint64_t d2 = pk(exp2i(e), exp2i(e)), inv2 = pk(exp2i(-e), exp2i(-e));
+                float L = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const uint64_t ap = pk(fabsf(x[2 * j]), fabsf(x[2 * j + 1]));
+                    float r0, r1;
+                    upk(mul2(ap, inv2), r0, r1);
+                    const uint64_t q2 = h2_to_f2(e2m1x2_round_h(r0, r1), neg_zero);
+                    const uint64_t e2 = sub2(ap, mul2_nofuse(q2, d2, z2));
+                    float s0, s1;
+                    upk(mul2_nofuse(e2, e2, z2), s0, s1);
+                    L = __fadd_rn(__fadd_rn(L, s0), s1);
+                }
+                if (first || L < best) { best = L; be = e; }
+                first = false;
+            }
+        }
+
+        // 3. emit the winner with its exact loss
         const float d = exp2i(be), inv = exp2i(-be);
-        uint32_t byte[16];
+        const uint64_t d2 = pk(d, d), inv2 = pk(inv, inv);
+        uint32_t word[4];
+        float L = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            byte[j] = e2m1x2(__fmul_rn(x[2 * j], inv), __fmul_rn(x[2 * j + 1], inv));
-        uint4 packed;
-        packed.x = byte[0] | byte[1] << 8 | byte[2] << 16 | byte[3] << 24;
-        packed.y = byte[4] | byte[5] << 8 | byte[6] << 16 | byte[7] << 24;
-        packed.z = byte[8] | byte[9] << 8 | byte[10] << 16 | byte[11] << 24;
-        packed.w = byte[12] | byte[13] << 8 | byte[14] << 16 | byte[15] << 24;
-        st_stream(codes + b * 16, packed);
-        scales[b] = (uint8_t)(be + 127);
-        if (loss) loss[b] = best;
-        if (deq) {
-            float y[32];
+        for (int c = 0; c < 4; ++c) {          // 8 elements per chunk: one 16-byte bf16 store
+            float y[8];
+            word[c] = 0;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                float qa, qb;
-                upk(e2m1x2_decode(byte[j]), qa, qb);
-                y[2 * j] = __fmul_rn(qa, d);
-                y[2 * j + 1] = __fmul_rn(qb, d);
+            for (int j = 0; j < 4; ++j) {
+                const int i = 8 * c + 2 * j;
+                const uint64_t xp = pk(x[i], x[i + 1]);
+                float r0, r1;
+                upk(mul2(xp, inv2), r0, r1);
+                const uint32_t byte = e2m1x2(r0, r1);
+                word[c] |= byte << (8 * j);
+                const uint64_t y2 = mul2_nofuse(h2_to_f2(e2m1x2_to_f16x2(byte), neg_zero), d2, z2);
+                upk(y2, y[2 * j], y[2 * j + 1]);
+                const uint64_t e2 = sub2(xp, y2);
+                float s0, s1;
+                upk(mul2_nofuse(e2, e2, z2), s0, s1);
+                L = __fadd_rn(__fadd_rn(L, s0), s1);
             }
-            store_block<32>(deq + b * 32, y);
+            if (deq) store_block<8>(deq + b * 32 + 8 * c, y);
         }
+#undef FP4Q_EK
+        st_stream(codes + b * 16, make_uint4(word[0], word[1], word[2], word[3]));
+        scales[b] = (uint8_t)(be + 127);
+        if (loss) loss[b] = L;
     }
 }
 

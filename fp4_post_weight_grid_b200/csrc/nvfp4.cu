@@ -31,6 +31,7 @@
 // so never wins a strict comparison, which keeps every lane on the same path.
 #include "device.cuh"
 #include "launch.h"
+#include "screen.cuh"
 
 namespace fp4q {
 
@@ -46,9 +47,8 @@ nvfp4_sweep_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_
                    float* __restrict__ d_S, T* __restrict__ deq, float* __restrict__ loss,
                    int32_t* __restrict__ d_status, float neg_zero)
 {
-    constexpr int NC = (NREAL + 1) & ~1;   // candidates evaluated in pairs
-    const uint64_t z2 = pk(neg_zero, neg_zero);
-    __shared__ float2 step[128];           // (d, inv) per E4M3 pattern
+    constexpr int NC = (NREAL + 1) & ~1;   // candidates screened in pairs
+    __shared__ float4 step[128];           // (d, inv, v^2, -) per E4M3 pattern
 
     const float gmax = __ldg(d_amax);
     const uint32_t gbits = __float_as_uint(gmax);
@@ -64,86 +64,139 @@ nvfp4_sweep_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_
     if (blockIdx.x == 0 && threadIdx.x == 0) *d_S = S;
     if (threadIdx.x < 128) {
         const uint32_t p = threadIdx.x == 0 ? 1u : (threadIdx.x == 127 ? 126u : threadIdx.x);
-        const float d = __fmul_rn(e4m3_value(p), S);
-        step[threadIdx.x] = make_float2(d, __frcp_rn(d));
+        const float v = e4m3_value(p);
+        const float d = __fmul_rn(v, S);
+        step[threadIdx.x] = make_float4(d, __frcp_rn(d), __fmul_rn(v, v), 0.0f);
     }
     __syncthreads();
     const float t6 = __fmul_rn(6.0f, S);
+    const float invS = 1.0f / S;                              // bound only
+    const float tS = 0x1p-70f * invS;
+    const float tau0 = tS * tS + 0x1p-120f;                   // subnormal allowance, S^2 units
+    const uint64_t z2 = pk(neg_zero, neg_zero);
 
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     for (int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x; b < nblocks; b += stride) {
         float x[16];
         load_block<16>(w + b * 16, x);
-        uint64_t aa[16];
-        float amax = 0.0f;
+        float amax = 0.0f, alpha2 = 0.0f;
+        float wt[16];
+        float tau = tau0;
+        bool prune = true;
+        if (WMSE) {
+            const float4* wp = reinterpret_cast<const float4*>(importance + (b % blocks_per_row) * 16);
+            uint32_t wbits = 0;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const float4 t = __ldg(wp + v);
+                wt[4 * v + 0] = t.x; wt[4 * v + 1] = t.y; wt[4 * v + 2] = t.z; wt[4 * v + 3] = t.w;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) wbits = max(wbits, __float_as_uint(wt[i]));
+            // the bound assumes 0 <= w <= 2^64 (sign bit clear, at most 2^64)
+            prune = wbits <= 0x5F800000u;
+            tau = tau0 * (1.0f + __uint_as_float(min(wbits, 0x5F800000u)));
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const float a = fabsf(x[i]);
             amax = fmaxf(amax, a);
-            aa[i] = pk(a, a);
+            const float as = a * invS;
+            alpha2 = WMSE ? fmaf(wt[i] * as, as, alpha2) : fmaf(as, as, alpha2);
         }
-        uint64_t ww[16];
-        if (WMSE) {
-            const float4* wp = reinterpret_cast<const float4*>(importance + (b % blocks_per_row) * 16);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const float4 t = __ldg(wp + v);
-                ww[4 * v + 0] = pk(t.x, t.x);
-                ww[4 * v + 1] = pk(t.y, t.y);
-                ww[4 * v + 2] = pk(t.z, t.z);
-                ww[4 * v + 3] = pk(t.w, t.w);
-            }
-        }
+        alpha2 *= 1.0f + 0x1p-16f;
         const int p = (int)e4m3_rn_sat(__fdiv_rn(amax, t6));   // s_base pattern
 
-        float best = 0.0f;
-        int bp = 1;
+        // 1. screen every candidate of the window
+        float lam[NC];
 #pragma unroll
         for (int k = 0; k < NC; k += 2) {
             const int pa = min(max(p + LO + min(k, NREAL - 1), 1), 126);
             const int pb = min(max(p + LO + min(k + 1, NREAL - 1), 1), 126);
-            const float2 sa = step[pa], sb = step[pb];
-            const uint64_t inv2 = pk(sa.y, sb.y), d2 = pk(sa.x, sb.x);
+            const float4 sa = step[pa], sb = step[pb];
+            const uint64_t inv2 = pk(sa.y, sb.y);
             uint64_t L2 = pk(0.0f, 0.0f);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
+                const float a = fabsf(x[i]);
                 float ra, rb;
-                upk(mul2(aa[i], inv2), ra, rb);
-                const uint64_t q2 = e2m1x2_round(ra, rb);
-                const uint64_t e2 = sub2(aa[i], mul2_nofuse(q2, d2, z2));
-                uint64_t s2 = mul2_nofuse(e2, e2, z2);
-                if (WMSE) s2 = mul2_nofuse(ww[i], s2, z2);
-                L2 = add2(L2, s2);
+                upk(mul2(pk(a, a), inv2), ra, rb);
+                const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
+                L2 = fma2(WMSE ? mul2(pk(wt[i], wt[i]), et) : et, et, L2);
             }
-            float La, Lb;
-            upk(L2, La, Lb);
-            if (k == 0 || La < best) { best = La; bp = pa; }
-            if (Lb < best) { best = Lb; bp = pb; }
+            upk(mul2(L2, pk(sa.z, sb.z)), lam[k], lam[k + 1]);
+        }
+        float M = lam[0];
+#pragma unroll
+        for (int k = 1; k < NREAL; ++k) M = fminf(M, lam[k]);
+        const float T = prune ? survivor_threshold(M, alpha2, tau) : __int_as_float(0x7F800000);
+        uint32_t mask = 0;
+#pragma unroll
+        for (int k = 0; k < NREAL; ++k) mask |= (lam[k] <= T ? 1u : 0u) << k;
+        if (mask == 0) mask = (1u << NREAL) - 1;   // unreachable for finite inputs; evaluate all
+
+        // 2. verify: exact loss of the survivors, first minimum wins
+        int bp;
+        if ((mask & (mask - 1)) == 0) {
+            bp = min(max(p + LO + __ffs(mask) - 1, 1), 126);
+        } else {
+            float best = 0.0f;
+            bool first = true;
+            bp = 1;
+            while (mask) {
+                const int k = __ffs(mask) - 1;
+                mask &= mask - 1;
+                const int pp = min(max(p + LO + k, 1), 126);
+                const float4 sc = step[pp];
+                const uint64_t d2 = pk(sc.x, sc.x), inv2 = pk(sc.y, sc.y);
+                float L = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint64_t ap = pk(fabsf(x[2 * j]), fabsf(x[2 * j + 1]));
+                    float r0, r1;
+                    upk(mul2(ap, inv2), r0, r1);
+                    const uint64_t q2 = h2_to_f2(e2m1x2_round_h(r0, r1), neg_zero);
+                    const uint64_t e2 = sub2(ap, mul2_nofuse(q2, d2, z2));
+                    uint64_t s2 = mul2_nofuse(e2, e2, z2);
+                    if (WMSE) s2 = mul2_nofuse(pk(wt[2 * j], wt[2 * j + 1]), s2, z2);
+                    float s0, s1;
+                    upk(s2, s0, s1);
+                    L = __fadd_rn(__fadd_rn(L, s0), s1);
+                }
+                if (first || L < best) { best = L; bp = pp; }
+                first = false;
+            }
         }
 
-        // emit the winner: codes from the signed values, reconstruction q*d
-        const float2 sw = step[bp];
+        // 3. emit the winner: codes from the signed values, reconstruction
+        //    q*d, and its exact loss
+        const float4 sw = step[bp];
+        const uint64_t d2 = pk(sw.x, sw.x), inv2 = pk(sw.y, sw.y);
         uint32_t byte[8];
+        float y[16];
+        float L = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            byte[j] = e2m1x2(__fmul_rn(x[2 * j], sw.y), __fmul_rn(x[2 * j + 1], sw.y));
+        for (int j = 0; j < 8; ++j) {
+            const uint64_t xp = pk(x[2 * j], x[2 * j + 1]);
+            float r0, r1;
+            upk(mul2(xp, inv2), r0, r1);
+            byte[j] = e2m1x2(r0, r1);
+            const uint64_t y2 = mul2_nofuse(h2_to_f2(e2m1x2_to_f16x2(byte[j]), neg_zero), d2, z2);
+            upk(y2, y[2 * j], y[2 * j + 1]);
+            const uint64_t e2 = sub2(xp, y2);
+            uint64_t s2 = mul2_nofuse(e2, e2, z2);
+            if (WMSE) s2 = mul2_nofuse(pk(wt[2 * j], wt[2 * j + 1]), s2, z2);
+            float s0, s1;
+            upk(s2, s0, s1);
+            L = __fadd_rn(__fadd_rn(L, s0), s1);
+        }
         uint2 packed;
         packed.x = byte[0] | byte[1] << 8 | byte[2] << 16 | byte[3] << 24;
         packed.y = byte[4] | byte[5] << 8 | byte[6] << 16 | byte[7] << 24;
         st_stream64(codes + b * 8, packed);
         scales[b] = (uint8_t)bp;
-        if (loss) loss[b] = best;
-        if (deq) {
-            float y[16];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float qa, qb;
-                upk(e2m1x2_decode(byte[j]), qa, qb);
-                y[2 * j] = __fmul_rn(qa, sw.x);
-                y[2 * j + 1] = __fmul_rn(qb, sw.x);
-            }
-            store_block<16>(deq + b * 16, y);
-        }
+        if (loss) loss[b] = L;
+        if (deq) store_block<16>(deq + b * 16, y);
     }
 }
 
