@@ -24,8 +24,9 @@ import torch
 __all__ = [
     "Fp4qError", "library_path", "load", "version", "check_status",
     "fp4q_global_absmax", "fp4q_nvfp4_sweepmse", "fp4q_nvfp4_sweepwmse", "fp4q_mxfp4_quant",
-    "fp4q_mxfp4_quant_hadamard", "fp4q_dequant", "fp4q_probe_e2m1", "fp4q_probe_e4m3",
-    "NVFP4Result", "MXFP4Result", "nvfp4_quantize", "mxfp4_quantize", "dequantize",
+    "fp4q_mxfp4_quant_hadamard", "fp4q_mxfp4_quant_absmax", "fp4q_quantize_dual", "fp4q_dequant",
+    "fp4q_probe_e2m1", "fp4q_probe_e4m3",
+    "NVFP4Result", "MXFP4Result", "nvfp4_quantize", "mxfp4_quantize", "quantize_dual", "dequantize",
     "FLAG_NONFINITE", "FLAG_RANGE",
 ]
 
@@ -40,7 +41,8 @@ FLAG_NONFINITE, FLAG_RANGE = 1, 2
 NVFP4_BLOCK, MXFP4_BLOCK = 16, 32
 EXPORTS = ("fp4q_version", "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_global_absmax",
            "fp4q_nvfp4_sweepmse", "fp4q_nvfp4_sweepwmse", "fp4q_mxfp4_quant",
-           "fp4q_mxfp4_quant_hadamard", "fp4q_dequant", "fp4q_probe_e2m1", "fp4q_probe_e4m3")
+           "fp4q_mxfp4_quant_hadamard", "fp4q_mxfp4_quant_absmax", "fp4q_quantize_dual", "fp4q_dequant",
+           "fp4q_probe_e2m1", "fp4q_probe_e4m3")
 
 
 class Fp4qError(RuntimeError):
@@ -79,6 +81,8 @@ def load():
         "fp4q_nvfp4_sweepwmse": [P, I, I64, I64, P, P, P, P, P, P, P, P, P],
         "fp4q_mxfp4_quant": [P, I, I64, I64, P, P, P, P, P, P],
         "fp4q_mxfp4_quant_hadamard": [P, I, I64, I64, P, P, P, P, P, P, P],
+        "fp4q_mxfp4_quant_absmax": [P, I, I64, I64, P, P, P, P, P, P, P, P],
+        "fp4q_quantize_dual": [P, I, I64, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, P],
         "fp4q_dequant": [I, P, P, P, I64, I64, P, I, P],
         "fp4q_probe_e2m1": [P, P, I64, P],
         "fp4q_probe_e4m3": [P, P, I64, P],
@@ -212,6 +216,29 @@ def fp4q_mxfp4_quant_hadamard(w, sign_masks, codes, scales, deq=None, block_loss
                                             _stream(stream)), "fp4q_mxfp4_quant_hadamard")
 
 
+def fp4q_mxfp4_quant_absmax(w, sign_masks, codes, scales, d_amax, deq=None, block_loss=None,
+                            d_status=None, stream=None) -> None:
+    """MXFP4 (rotated when sign_masks is given) that also writes max|w| to d_amax."""
+    rows, cols, wp, cp, sp, dp, lp, st = _mx_args(w, codes, scales, deq, block_loss, d_status)
+    mp = _dev(sign_masks, "sign_masks", (torch.int32, torch.uint32), cols // MXFP4_BLOCK, w.device)
+    ap = _dev(d_amax, "d_amax", torch.float32, 1, w.device)
+    _check(load().fp4q_mxfp4_quant_absmax(wp, _wdtype(w), rows, cols, mp, cp, sp, dp, lp, ap, st,
+                                          _stream(stream)), "fp4q_mxfp4_quant_absmax")
+
+
+def fp4q_quantize_dual(w, importance, sign_masks, d_amax, nv_codes, nv_scales, d_global_scale,
+                       nv_deq, nv_loss, mx_codes, mx_scales, mx_deq, mx_loss, d_status,
+                       stream=None) -> None:
+    """NVFP4 ScaleSweep and MXFP4 of the same weight in two launches."""
+    rows, cols, wp, cp, sp, dp, lp, st = _mx_args(w, mx_codes, mx_scales, mx_deq, mx_loss, d_status)
+    _, _, _, ap, ncp, nsp, gp, ndp, nlp, _ = _nvfp4_args(w, d_amax, nv_codes, nv_scales, d_global_scale,
+                                                        nv_deq, nv_loss, d_status)
+    ip = _dev(importance, "importance", torch.float32, cols, w.device)
+    mp = _dev(sign_masks, "sign_masks", (torch.int32, torch.uint32), cols // MXFP4_BLOCK, w.device)
+    _check(load().fp4q_quantize_dual(wp, _wdtype(w), rows, cols, ip, mp, ap, ncp, nsp, gp, ndp, nlp,
+                                     cp, sp, dp, lp, st, _stream(stream)), "fp4q_quantize_dual")
+
+
 def fp4q_dequant(fmt: int, codes, scales, d_global_scale, rows: int, cols: int, out,
                  stream=None) -> None:
     """Decode codes + scales (+ S for NVFP4) into `out` (bf16 or fp32)."""
@@ -296,6 +323,31 @@ def mxfp4_quantize(w: torch.Tensor, sign_masks: Optional[torch.Tensor] = None, w
     else:
         fp4q_mxfp4_quant_hadamard(w, sign_masks, codes, scales, deq, loss, status, stream)
     return MXFP4Result(codes, scales, deq, loss, status)
+
+
+def quantize_dual(w: torch.Tensor, importance: Optional[torch.Tensor] = None,
+                  sign_masks: Optional[torch.Tensor] = None, with_deq=True, with_loss=True,
+                  stream=None):
+    """NVFP4 (MSE, or WMSE with `importance`) and MXFP4 (rotated with `sign_masks`)
+    of the same weight; returns (NVFP4Result, MXFP4Result) sharing one status word."""
+    rows, cols = _rc(w, MXFP4_BLOCK)
+    dev = w.device
+    amax = torch.empty(1, dtype=torch.float32, device=dev)
+    S = torch.empty(1, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    nv = NVFP4Result(torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+                     torch.empty((rows, cols // NVFP4_BLOCK), dtype=torch.uint8, device=dev), S,
+                     torch.empty_like(w) if with_deq else None,
+                     torch.empty((rows, cols // NVFP4_BLOCK), dtype=torch.float32, device=dev) if with_loss else None,
+                     amax, status)
+    mx = MXFP4Result(torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+                     torch.empty((rows, cols // MXFP4_BLOCK), dtype=torch.uint8, device=dev),
+                     torch.empty_like(w) if with_deq else None,
+                     torch.empty((rows, cols // MXFP4_BLOCK), dtype=torch.float32, device=dev) if with_loss else None,
+                     status)
+    fp4q_quantize_dual(w, importance, sign_masks, amax, nv.codes, nv.scales, S, nv.deq, nv.block_loss,
+                       mx.codes, mx.scales, mx.deq, mx.block_loss, status, stream)
+    return nv, mx
 
 
 def dequantize(fmt: int, codes: torch.Tensor, scales: torch.Tensor, global_scale=None,

@@ -2,6 +2,9 @@
 // stream-ordered launch per call.  No allocation, no host synchronization.
 #include <cstdint>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include <cuda_runtime.h>
 
@@ -20,6 +23,24 @@ int sm_count()
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
     if (dev < 64) cached[dev] = n;
     return n;
+}
+
+int resident_blocks_per_sm(const void* kernel, int threads, size_t dyn_smem)
+{
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, int> cache;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find({kernel, dev});
+    if (it != cache.end()) return it->second;
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, dyn_smem) != cudaSuccess ||
+        per_sm <= 0)
+        per_sm = 1;
+    cache[{kernel, dev}] = per_sm;
+    return per_sm;
 }
 
 }  // namespace fp4q
@@ -147,7 +168,7 @@ static fp4q_status mxfp4_common(const void* w, fp4q_dtype dt, int64_t rows, int6
     if (rotate && !masks) return FP4Q_ERR_NULL;
     if (rotate && !aligned(masks, 4)) return FP4Q_ERR_ALIGN;
     fp4q::launch_mxfp4(w, dt == FP4Q_BF16, rows, cols, rotate ? masks : nullptr, codes, scales, deq,
-                       loss, d_status, reinterpret_cast<cudaStream_t>(stream));
+                       loss, d_status, nullptr, reinterpret_cast<cudaStream_t>(stream));
     return after_launch();
 }
 
@@ -166,6 +187,51 @@ fp4q_status fp4q_mxfp4_quant_hadamard(const void* w, fp4q_dtype dt, int64_t rows
 {
     return mxfp4_common(w, dt, rows, cols, sign_masks, true, codes, scales_e8m0, deq, block_loss,
                         d_status, stream);
+}
+
+fp4q_status fp4q_mxfp4_quant_absmax(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                    const uint32_t* sign_masks, uint8_t* codes, uint8_t* scales_e8m0,
+                                    void* deq, float* block_loss, float* d_amax, int32_t* d_status,
+                                    fp4q_stream_t stream)
+{
+    if (!valid_dtype(dt)) return FP4Q_ERR_DTYPE;
+    if (!shape_ok(rows, cols, FP4Q_MXFP4_BLOCK)) return FP4Q_ERR_SHAPE;
+    if (!d_amax) return FP4Q_ERR_NULL;
+    if (!aligned(d_amax, 4)) return FP4Q_ERR_ALIGN;
+    if (rows == 0 || cols == 0) {      // max over no elements: 0
+        cudaMemsetAsync(d_amax, 0, sizeof(float), reinterpret_cast<cudaStream_t>(stream));
+        return after_launch();
+    }
+    bool empty = false;
+    fp4q_status st = check_quant_args(w, dt, rows, cols, FP4Q_MXFP4_BLOCK, codes, scales_e8m0, d_status,
+                                      deq, block_loss, 16, &empty);
+    if (st != FP4Q_OK) return st;
+    if (sign_masks && !aligned(sign_masks, 4)) return FP4Q_ERR_ALIGN;
+    fp4q::launch_mxfp4(w, dt == FP4Q_BF16, rows, cols, sign_masks, codes, scales_e8m0, deq, block_loss,
+                       d_status, d_amax, reinterpret_cast<cudaStream_t>(stream));
+    return after_launch();
+}
+
+fp4q_status fp4q_quantize_dual(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                               const float* importance, const uint32_t* sign_masks, float* d_amax,
+                               uint8_t* nv_codes, uint8_t* nv_scales, float* d_global_scale,
+                               void* nv_deq, float* nv_loss, uint8_t* mx_codes, uint8_t* mx_scales,
+                               void* mx_deq, float* mx_loss, int32_t* d_status, fp4q_stream_t stream)
+{
+    bool empty = false;
+    fp4q_status st = check_quant_args(w, dt, rows, cols, FP4Q_MXFP4_BLOCK, nv_codes, nv_scales,
+                                      d_status, nv_deq, nv_loss, 8, &empty);
+    if (st != FP4Q_OK) return st;
+    if (!d_amax || !d_global_scale) return FP4Q_ERR_NULL;
+    if (!aligned(d_amax, 4) || !aligned(d_global_scale, 4) || (importance && !aligned(importance, 16)))
+        return FP4Q_ERR_ALIGN;
+    if (empty) return fp4q_mxfp4_quant_absmax(w, dt, rows, cols, sign_masks, mx_codes, mx_scales,
+                                              mx_deq, mx_loss, d_amax, d_status, stream);
+    st = fp4q_mxfp4_quant_absmax(w, dt, rows, cols, sign_masks, mx_codes, mx_scales, mx_deq, mx_loss,
+                                 d_amax, d_status, stream);
+    if (st != FP4Q_OK) return st;
+    return nvfp4_common(w, dt, rows, cols, d_amax, importance, importance != nullptr, nv_codes, nv_scales,
+                        d_global_scale, nv_deq, nv_loss, d_status, stream);
 }
 
 fp4q_status fp4q_dequant(fp4q_format format, const uint8_t* codes, const uint8_t* scales,

@@ -10,6 +10,26 @@ namespace fp4q {
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
+// Resident thread blocks per SM of `kernel` with `threads` threads and
+// `dyn_smem` bytes of dynamic shared memory on the current device; raises the
+// kernel's dynamic shared memory limit the first time.  Cached per (kernel,
+// device).
+int resident_blocks_per_sm(const void* kernel, int threads, size_t dyn_smem);
+
+// Grid for a grid-stride kernel: the work is split into equal shares for about
+// two generations of resident thread blocks (a thread block that finishes early
+// is replaced, which evens out the tail), never more blocks than the work needs.
+template <typename Kernel>
+inline int64_t resident_grid(Kernel kernel, int threads, size_t dyn_smem, int64_t work_items)
+{
+    const int per_sm = resident_blocks_per_sm(reinterpret_cast<const void*>(kernel), threads, dyn_smem);
+    const int64_t per_gen = (int64_t)per_sm * sm_count() * threads * 2;
+    const int64_t rounds = (work_items + per_gen - 1) / per_gen;
+    const int64_t share = rounds < 1 ? 1 : rounds;
+    const int64_t g = (work_items + threads * share - 1) / (threads * share);
+    return g < 1 ? 1 : g;
+}
+
 void launch_absmax(const void* x, bool bf16, int64_t n, float* d_amax, cudaStream_t s);
 
 // NVFP4 ScaleSweep: importance == nullptr selects MSE (window -3..+7), otherwise
@@ -18,10 +38,11 @@ void launch_nvfp4_sweep(const void* w, bool bf16, int64_t rows, int64_t cols, co
                         const float* importance, uint8_t* codes, uint8_t* scales, float* d_S,
                         void* deq, float* loss, int32_t* d_status, cudaStream_t s);
 
-// MXFP4 with the E8M0 e0-1..e0+1 sweep; sign_masks != nullptr adds the block Hadamard.
+// MXFP4 with the E8M0 e0-1..e0+1 sweep; sign_masks != nullptr adds the block
+// Hadamard; d_amax != nullptr also writes max|w| of the unrotated input there.
 void launch_mxfp4(const void* w, bool bf16, int64_t rows, int64_t cols, const uint32_t* sign_masks,
                   uint8_t* codes, uint8_t* scales, void* deq, float* loss, int32_t* d_status,
-                  cudaStream_t s);
+                  float* d_amax, cudaStream_t s);
 
 void launch_dequant(bool mx, const uint8_t* codes, const uint8_t* scales, const float* d_S,
                     int64_t rows, int64_t cols, void* out, bool out_bf16, cudaStream_t s);

@@ -31,18 +31,26 @@ namespace {
 constexpr int kThreads = 256;
 constexpr float kInvSqrt32 = 0x1.6a09e6p-3f;   // RN(1/sqrt(32))
 
-template <typename T, bool HAD>
-__global__ void __launch_bounds__(kThreads)
+// AMAX: also reduce max|w| of the unrotated input into *gmax_bits (an atomic
+// max on the binary32 bit pattern, which keeps NaN and Inf), for the NVFP4
+// global scale of the same weight.
+template <typename T, bool HAD, bool AMAX>
+__global__ void __launch_bounds__(kThreads, 3)
 mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
              const uint32_t* __restrict__ masks, uint8_t* __restrict__ codes,
              uint8_t* __restrict__ scales, T* __restrict__ deq, float* __restrict__ loss,
-             int32_t* __restrict__ d_status, float neg_zero)
+             int32_t* __restrict__ d_status, float neg_zero, unsigned* __restrict__ gmax_bits)
 {
     const uint64_t z2 = pk(neg_zero, neg_zero);
+    uint32_t wmax = 0;     // AMAX: max |w| bits over this thread's blocks
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     for (int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x; b < nblocks; b += stride) {
         float x[32];
         load_block<32>(w + b * 32, x);
+        if (HAD && AMAX) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) wmax = max(wmax, __float_as_uint(x[j]) & 0x7FFFFFFFu);
+        }
         if (HAD) {
             const uint32_t m = __ldg(masks + (b % blocks_per_row));
 #pragma unroll
@@ -61,10 +69,15 @@ mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
 #pragma unroll
             for (int j = 0; j < 32; ++j) x[j] = __fmul_rn(x[j], kInvSqrt32);
         }
+        float a[32];        // |y|, shared by every stage below
         uint32_t abits = 0;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) abits = max(abits, __float_as_uint(x[j]) & 0x7FFFFFFFu);
+        for (int j = 0; j < 32; ++j) {
+            a[j] = fabsf(x[j]);
+            abits = max(abits, __float_as_uint(a[j]));
+        }
         if (abits >= 0x7F800000u) atomicOr(d_status, kFlagNonfinite);
+        if (!HAD && AMAX) wmax = max(wmax, abits);
         int e0 = -127;
         if (abits >= 0x00800000u) {
             const int a = (int)(abits >> 23) - 127;                 // floor(log2 amax)
@@ -76,30 +89,50 @@ mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
 
         // 1. screen the three exponents in units of 2^e0 (S = 2^e0, v = 2^(e-e0))
         const float inv0 = exp2i(-e0);
-        float alpha2 = 0.0f;
+        float alpha2;
+        {
+            uint64_t al2 = pk(0.0f, 0.0f);
+            const uint64_t inv02 = pk(inv0, inv0);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const float as = fabsf(x[j]) * inv0;
-            alpha2 = fmaf(as, as, alpha2);
+            for (int j = 0; j < 16; ++j) {
+                const uint64_t as = mul2(pk(a[2 * j], a[2 * j + 1]), inv02);
+                al2 = fma2(as, as, al2);
+            }
+            float lo, hi;
+            upk(al2, lo, hi);
+            alpha2 = (lo + hi) * (1.0f + 0x1p-16f);   // bound only: rounded up generously
         }
-        alpha2 *= 1.0f + 0x1p-16f;
         const float tS = 0x1p-70f * inv0;
         const float tau = tS * tS + 0x1p-120f;
-        float lam[4];
-#pragma unroll
-        for (int k = 0; k < 4; k += 2) {
-            const int ea = FP4Q_EK(k), eb = FP4Q_EK(min(k + 1, 2));
+        float lam[3];
+        {   // exponents e0-1 and e0 as a pair, one element at a time
+            const int ea = FP4Q_EK(0), eb = FP4Q_EK(1);
             const uint64_t inv2 = pk(exp2i(-ea), exp2i(-eb));
             uint64_t L2 = pk(0.0f, 0.0f);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float a = fabsf(x[i]);
                 float ra, rb;
-                upk(mul2(pk(a, a), inv2), ra, rb);
+                upk(mul2(pk(a[i], a[i]), inv2), ra, rb);
                 const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
                 L2 = fma2(et, et, L2);
             }
-            upk(mul2(L2, pk(exp2i(2 * (ea - e0)), exp2i(2 * (eb - e0)))), lam[k], lam[k + 1]);
+            upk(mul2(L2, pk(exp2i(2 * (ea - e0)), exp2i(2 * (eb - e0)))), lam[0], lam[1]);
+        }
+        {   // exponent e0+1, two elements at a time
+            const int ec = FP4Q_EK(2);
+            const float invc = exp2i(-ec);
+            const uint64_t inv2 = pk(invc, invc);
+            uint64_t L2 = pk(0.0f, 0.0f);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                float ra, rb;
+                upk(mul2(pk(a[2 * j], a[2 * j + 1]), inv2), ra, rb);
+                const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
+                L2 = fma2(et, et, L2);
+            }
+            float lo, hi;
+            upk(L2, lo, hi);
+            lam[2] = (lo + hi) * exp2i(2 * (ec - e0));
         }
         const float M = fminf(fminf(lam[0], lam[1]), lam[2]);
         const float T = survivor_threshold(M, alpha2, tau);
@@ -122,7 +155,7 @@ mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
                 float L = 0.0f;
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const uint64_t ap = pk(fabsf(x[2 * j]), fabsf(x[2 * j + 1]));
+                    const uint64_t ap = pk(a[2 * j], a[2 * j + 1]);
                     float r0, r1;
                     upk(mul2(ap, inv2), r0, r1);
                     const uint64_t q2 = h2_to_f2(e2m1x2_round_h(r0, r1), neg_zero);
@@ -155,10 +188,12 @@ mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
                 word[c] |= byte << (8 * j);
                 const uint64_t y2 = mul2_nofuse(h2_to_f2(e2m1x2_to_f16x2(byte), neg_zero), d2, z2);
                 upk(y2, y[2 * j], y[2 * j + 1]);
-                const uint64_t e2 = sub2(xp, y2);
-                float s0, s1;
-                upk(mul2_nofuse(e2, e2, z2), s0, s1);
-                L = __fadd_rn(__fadd_rn(L, s0), s1);
+                if (loss) {     // the winner is known; its exact loss is only an output
+                    const uint64_t e2 = sub2(xp, y2);
+                    float s0, s1;
+                    upk(mul2_nofuse(e2, e2, z2), s0, s1);
+                    L = __fadd_rn(__fadd_rn(L, s0), s1);
+                }
             }
             if (deq) store_block<8>(deq + b * 32 + 8 * c, y);
         }
@@ -167,40 +202,60 @@ mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
         scales[b] = (uint8_t)(be + 127);
         if (loss) loss[b] = L;
     }
+    if (AMAX) {
+        __shared__ uint32_t warp_max[kThreads / 32];
+        wmax = __reduce_max_sync(0xFFFFFFFFu, wmax);
+        if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = wmax;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            wmax = threadIdx.x < kThreads / 32 ? warp_max[threadIdx.x] : 0u;
+            wmax = __reduce_max_sync(0xFFFFFFFFu, wmax);
+            if (threadIdx.x == 0 && wmax != 0u) atomicMax(gmax_bits, wmax);
+        }
+    }
 }
 
-template <typename T, bool HAD>
+template <typename T, bool HAD, bool AMAX>
 void launch_typed(const void* w, int64_t rows, int64_t cols, const uint32_t* masks, uint8_t* codes,
-                  uint8_t* scales, void* deq, float* loss, int32_t* d_status, cudaStream_t s)
+                  uint8_t* scales, void* deq, float* loss, int32_t* d_status, unsigned* gmax_bits,
+                  cudaStream_t s)
 {
     const int64_t nblocks = rows * (cols / 32);
-    const int64_t per_wave = (int64_t)sm_count() * 8 * kThreads;
-    const int64_t waves = (nblocks + per_wave - 1) / per_wave;
-    int64_t grid = (nblocks + kThreads * waves - 1) / (kThreads * waves);
-    if (grid < 1) grid = 1;
-    mxfp4_kernel<T, HAD><<<(unsigned)grid, kThreads, 0, s>>>(
+    const int64_t grid = resident_grid(mxfp4_kernel<T, HAD, AMAX>, kThreads, 0, nblocks);
+    mxfp4_kernel<T, HAD, AMAX><<<(unsigned)grid, kThreads, 0, s>>>(
         static_cast<const T*>(w), nblocks, cols / 32, masks, codes, scales, static_cast<T*>(deq),
-        loss, d_status, -0.0f);
+        loss, d_status, -0.0f, gmax_bits);
+}
+
+template <typename T, bool AMAX>
+void launch_rot(const void* w, int64_t rows, int64_t cols, const uint32_t* masks, uint8_t* codes,
+                uint8_t* scales, void* deq, float* loss, int32_t* d_status, unsigned* gmax_bits,
+                cudaStream_t s)
+{
+    if (masks)
+        launch_typed<T, true, AMAX>(w, rows, cols, masks, codes, scales, deq, loss, d_status, gmax_bits, s);
+    else
+        launch_typed<T, false, AMAX>(w, rows, cols, nullptr, codes, scales, deq, loss, d_status, gmax_bits, s);
 }
 
 }  // namespace
 
 void launch_mxfp4(const void* w, bool bf16, int64_t rows, int64_t cols, const uint32_t* sign_masks,
                   uint8_t* codes, uint8_t* scales, void* deq, float* loss, int32_t* d_status,
-                  cudaStream_t s)
+                  float* d_amax, cudaStream_t s)
 {
-    if (sign_masks) {
+    unsigned* g = reinterpret_cast<unsigned*>(d_amax);
+    if (d_amax) {
+        cudaMemsetAsync(d_amax, 0, sizeof(float), s);
         if (bf16)
-            launch_typed<__nv_bfloat16, true>(w, rows, cols, sign_masks, codes, scales, deq, loss,
-                                              d_status, s);
+            launch_rot<__nv_bfloat16, true>(w, rows, cols, sign_masks, codes, scales, deq, loss, d_status, g, s);
         else
-            launch_typed<float, true>(w, rows, cols, sign_masks, codes, scales, deq, loss, d_status, s);
+            launch_rot<float, true>(w, rows, cols, sign_masks, codes, scales, deq, loss, d_status, g, s);
     } else {
         if (bf16)
-            launch_typed<__nv_bfloat16, false>(w, rows, cols, nullptr, codes, scales, deq, loss,
-                                               d_status, s);
+            launch_rot<__nv_bfloat16, false>(w, rows, cols, sign_masks, codes, scales, deq, loss, d_status, g, s);
         else
-            launch_typed<float, false>(w, rows, cols, nullptr, codes, scales, deq, loss, d_status, s);
+            launch_rot<float, false>(w, rows, cols, sign_masks, codes, scales, deq, loss, d_status, g, s);
     }
 }
 

@@ -47,8 +47,14 @@ nvfp4_sweep_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_
                    float* __restrict__ d_S, T* __restrict__ deq, float* __restrict__ loss,
                    int32_t* __restrict__ d_status, float neg_zero)
 {
-    constexpr int NC = (NREAL + 1) & ~1;   // candidates screened in pairs
-    __shared__ float4 step[128];           // (d, inv, v^2, -) per E4M3 pattern
+    constexpr int NC = (NREAL + 1) & ~1;
+    // Per E4M3 pattern: (d, inv, v^2); then, for every window position j = p' + 8
+    // (p' = p + LO + 2k may run from -8 to 140), the pairs (inv[p'], inv[p'+1])
+    // and (v^2[p'], v^2[p'+1]) with each pattern clipped to 0x01..0x7E, so that
+    // one aligned 8-byte shared load yields a candidate pair's operands.
+    constexpr int kPairs = 152, kOff = 8;
+    __shared__ float4 step[128];
+    __shared__ float2 inv_pair[kPairs], vsq_pair[kPairs];
 
     const float gmax = __ldg(d_amax);
     const uint32_t gbits = __float_as_uint(gmax);
@@ -67,6 +73,13 @@ nvfp4_sweep_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_
         const float v = e4m3_value(p);
         const float d = __fmul_rn(v, S);
         step[threadIdx.x] = make_float4(d, __frcp_rn(d), __fmul_rn(v, v), 0.0f);
+    }
+    __syncthreads();
+    if (threadIdx.x < kPairs) {
+        const int pa = min(max((int)threadIdx.x - kOff, 1), 126);
+        const int pb = min(max((int)threadIdx.x - kOff + 1, 1), 126);
+        inv_pair[threadIdx.x] = make_float2(step[pa].y, step[pb].y);
+        vsq_pair[threadIdx.x] = make_float2(step[pa].z, step[pb].z);
     }
     __syncthreads();
     const float t6 = __fmul_rn(6.0f, S);
@@ -97,34 +110,66 @@ nvfp4_sweep_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_
             prune = wbits <= 0x5F800000u;
             tau = tau0 * (1.0f + __uint_as_float(min(wbits, 0x5F800000u)));
         }
+        float a[16];        // |x|, shared by every stage below
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float a = fabsf(x[i]);
-            amax = fmaxf(amax, a);
-            const float as = a * invS;
-            alpha2 = WMSE ? fmaf(wt[i] * as, as, alpha2) : fmaf(as, as, alpha2);
+        for (int i = 0; i < 16; ++i) a[i] = fabsf(x[i]);
+        uint64_t al2 = pk(0.0f, 0.0f);
+        const uint64_t invS2 = pk(invS, invS);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            amax = fmaxf(amax, fmaxf(a[2 * j], a[2 * j + 1]));
+            const uint64_t as = mul2(pk(a[2 * j], a[2 * j + 1]), invS2);
+            al2 = fma2(WMSE ? mul2(pk(wt[2 * j], wt[2 * j + 1]), as) : as, as, al2);
         }
-        alpha2 *= 1.0f + 0x1p-16f;
+        {
+            float lo, hi;
+            upk(al2, lo, hi);
+            alpha2 = (lo + hi) * (1.0f + 0x1p-16f);   // bound only: rounded up generously
+        }
         const int p = (int)e4m3_rn_sat(__fdiv_rn(amax, t6));   // s_base pattern
 
         // 1. screen every candidate of the window
+        constexpr int NP = NREAL / 2;          // candidate pairs screened together
         float lam[NC];
+        {
+            uint64_t inv2[NP], L2[NP];
+            const uint64_t* invp = reinterpret_cast<const uint64_t*>(inv_pair) + (p + LO + kOff);
 #pragma unroll
-        for (int k = 0; k < NC; k += 2) {
-            const int pa = min(max(p + LO + min(k, NREAL - 1), 1), 126);
-            const int pb = min(max(p + LO + min(k + 1, NREAL - 1), 1), 126);
-            const float4 sa = step[pa], sb = step[pb];
-            const uint64_t inv2 = pk(sa.y, sb.y);
+            for (int k = 0; k < NP; ++k) {
+                inv2[k] = invp[2 * k];
+                L2[k] = pk(0.0f, 0.0f);
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {     // element outer: the (|x|, |x|) pair is built once
+                const uint64_t aa = pk(a[i], a[i]);
+                const uint64_t w2 = WMSE ? pk(wt[i], wt[i]) : 0;
+#pragma unroll
+                for (int k = 0; k < NP; ++k) {
+                    float ra, rb;
+                    upk(mul2(aa, inv2[k]), ra, rb);
+                    const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
+                    L2[k] = fma2(WMSE ? mul2(w2, et) : et, et, L2[k]);
+                }
+            }
+            const uint64_t* vsqp = reinterpret_cast<const uint64_t*>(vsq_pair) + (p + LO + kOff);
+#pragma unroll
+            for (int k = 0; k < NP; ++k) upk(mul2(L2[k], vsqp[2 * k]), lam[2 * k], lam[2 * k + 1]);
+        }
+        if (NREAL & 1) {    // the odd last candidate, two elements per packed operation
+            const float il = inv_pair[p + LO + NREAL - 1 + kOff].x;
+            const float vl = vsq_pair[p + LO + NREAL - 1 + kOff].x;
+            const uint64_t inv2 = pk(il, il);
             uint64_t L2 = pk(0.0f, 0.0f);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float a = fabsf(x[i]);
+            for (int j = 0; j < 8; ++j) {
                 float ra, rb;
-                upk(mul2(pk(a, a), inv2), ra, rb);
+                upk(mul2(pk(a[2 * j], a[2 * j + 1]), inv2), ra, rb);
                 const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
-                L2 = fma2(WMSE ? mul2(pk(wt[i], wt[i]), et) : et, et, L2);
+                L2 = fma2(WMSE ? mul2(pk(wt[2 * j], wt[2 * j + 1]), et) : et, et, L2);
             }
-            upk(mul2(L2, pk(sa.z, sb.z)), lam[k], lam[k + 1]);
+            float lo, hi;
+            upk(L2, lo, hi);
+            lam[NREAL - 1] = (lo + hi) * vl;
         }
         float M = lam[0];
 #pragma unroll
@@ -152,7 +197,7 @@ nvfp4_sweep_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_
                 float L = 0.0f;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const uint64_t ap = pk(fabsf(x[2 * j]), fabsf(x[2 * j + 1]));
+                    const uint64_t ap = pk(a[2 * j], a[2 * j + 1]);
                     float r0, r1;
                     upk(mul2(ap, inv2), r0, r1);
                     const uint64_t q2 = h2_to_f2(e2m1x2_round_h(r0, r1), neg_zero);
@@ -183,12 +228,14 @@ nvfp4_sweep_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_
             byte[j] = e2m1x2(r0, r1);
             const uint64_t y2 = mul2_nofuse(h2_to_f2(e2m1x2_to_f16x2(byte[j]), neg_zero), d2, z2);
             upk(y2, y[2 * j], y[2 * j + 1]);
-            const uint64_t e2 = sub2(xp, y2);
-            uint64_t s2 = mul2_nofuse(e2, e2, z2);
-            if (WMSE) s2 = mul2_nofuse(pk(wt[2 * j], wt[2 * j + 1]), s2, z2);
-            float s0, s1;
-            upk(s2, s0, s1);
-            L = __fadd_rn(__fadd_rn(L, s0), s1);
+            if (loss) {     // the winner is known; its exact loss is only an output
+                const uint64_t e2 = sub2(xp, y2);
+                uint64_t s2 = mul2_nofuse(e2, e2, z2);
+                if (WMSE) s2 = mul2_nofuse(pk(wt[2 * j], wt[2 * j + 1]), s2, z2);
+                float s0, s1;
+                upk(s2, s0, s1);
+                L = __fadd_rn(__fadd_rn(L, s0), s1);
+            }
         }
         uint2 packed;
         packed.x = byte[0] | byte[1] << 8 | byte[2] << 16 | byte[3] << 24;
@@ -206,11 +253,7 @@ void launch_typed(const void* w, int64_t rows, int64_t cols, const float* d_amax
                   void* deq, float* loss, int32_t* d_status, cudaStream_t s)
 {
     const int64_t nblocks = rows * (cols / 16);
-    // balanced waves of at most 8 resident thread blocks per SM
-    const int64_t per_wave = (int64_t)sm_count() * 8 * kThreads;
-    const int64_t waves = (nblocks + per_wave - 1) / per_wave;
-    int64_t grid = (nblocks + kThreads * waves - 1) / (kThreads * waves);
-    if (grid < 1) grid = 1;
+    const int64_t grid = resident_grid(nvfp4_sweep_kernel<T, LO, NREAL, WMSE>, kThreads, 0, nblocks);
     nvfp4_sweep_kernel<T, LO, NREAL, WMSE><<<(unsigned)grid, kThreads, 0, s>>>(
         static_cast<const T*>(w), nblocks, cols / 16, d_amax, importance, codes, scales, d_S,
         static_cast<T*>(deq), loss, d_status, -0.0f);

@@ -104,13 +104,14 @@ __device__ __forceinline__ uint32_t e2m1x2_round_h(float lo, float hi)
 // mixed-precision subtracts (each one rounding; the f16 operand is exact).
 __device__ __forceinline__ uint64_t sub_h2_f2(uint32_t q2, float rlo, float rhi)
 {
-    float a, b;
-    asm("{\n\t.reg .f16 l, h;\n\t"
-        "mov.b32 {l, h}, %2;\n\t"
-        "sub.rn.f32.f16 %0, l, %3;\n\t"
-        "sub.rn.f32.f16 %1, h, %4;\n\t}"
-        : "=f"(a), "=f"(b) : "r"(q2), "f"(rlo), "f"(rhi));
-    return pk(a, b);
+    uint64_t r;    // the two results are formed in place as one register pair
+    asm("{\n\t.reg .f16 l, h;\n\t.reg .f32 a, b;\n\t"
+        "mov.b32 {l, h}, %1;\n\t"
+        "sub.rn.f32.f16 a, l, %2;\n\t"
+        "sub.rn.f32.f16 b, h, %3;\n\t"
+        "mov.b64 %0, {a, b};\n\t}"
+        : "=l"(r) : "r"(q2), "f"(rlo), "f"(rhi));
+    return r;
 }
 
 // Exact binary32 value of an f16x2 pair, via mixed adds of -0 (exact; the
@@ -118,13 +119,14 @@ __device__ __forceinline__ uint64_t sub_h2_f2(uint32_t q2, float rlo, float rhi)
 // -0.0f so that the adds are not folded away.
 __device__ __forceinline__ uint64_t h2_to_f2(uint32_t q2, float nz)
 {
-    float a, b;
-    asm("{\n\t.reg .f16 l, h;\n\t"
-        "mov.b32 {l, h}, %2;\n\t"
-        "add.rn.f32.f16 %0, l, %3;\n\t"
-        "add.rn.f32.f16 %1, h, %3;\n\t}"
-        : "=f"(a), "=f"(b) : "r"(q2), "f"(nz));
-    return pk(a, b);
+    uint64_t r;
+    asm("{\n\t.reg .f16 l, h;\n\t.reg .f32 a, b;\n\t"
+        "mov.b32 {l, h}, %1;\n\t"
+        "add.rn.f32.f16 a, l, %2;\n\t"
+        "add.rn.f32.f16 b, h, %2;\n\t"
+        "mov.b64 %0, {a, b};\n\t}"
+        : "=l"(r) : "r"(q2), "f"(nz));
+    return r;
 }
 
 __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)

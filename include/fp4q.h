@@ -195,6 +195,42 @@ fp4q_status fp4q_mxfp4_quant_hadamard(const void* w, fp4q_dtype dt, int64_t rows
                                       int32_t* d_status, fp4q_stream_t stream);
 
 /*
+ * fp4q_mxfp4_quant_absmax -- fp4q_mxfp4_quant (sign_masks == NULL) or
+ * fp4q_mxfp4_quant_hadamard (sign_masks != NULL) that also writes max|w| of
+ * the unrotated weight to *d_amax, exactly as fp4q_global_absmax would (NaN
+ * and Inf propagate), so that an NVFP4 sweep of the same weight needs no
+ * separate read for its global scale ("Metodologia: ScaleSweep" sec. 2).
+ *   d_amax  device float, overwritten (zeroed first, then atomic max).
+ * Other arguments and errors as fp4q_mxfp4_quant; an empty tensor only
+ * zeroes *d_amax.
+ */
+fp4q_status fp4q_mxfp4_quant_absmax(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                    const uint32_t* sign_masks, uint8_t* codes, uint8_t* scales_e8m0,
+                                    void* deq, float* block_loss, float* d_amax, int32_t* d_status,
+                                    fp4q_stream_t stream);
+
+/*
+ * fp4q_quantize_dual -- NVFP4 ScaleSweep and MXFP4 of the same weight.
+ * The same results as fp4q_global_absmax + fp4q_nvfp4_sweep{mse,wmse} +
+ * fp4q_mxfp4_quant{,_hadamard}, in two launches instead of three:
+ * fp4q_mxfp4_quant_absmax, then the NVFP4 sweep (MSE when importance is NULL,
+ * WMSE otherwise) on its *d_amax, so W is read twice instead of three times.
+ *   importance  device or NULL (cols floats, 16-byte aligned): WMSE weights.
+ *   sign_masks  device or NULL (cols/32 uint32): rotate the MXFP4 blocks.
+ *   d_amax, d_global_scale  device floats (written).
+ *   nv_*        NVFP4 outputs as in fp4q_nvfp4_sweepmse (nv_deq, nv_loss
+ *               may be NULL).
+ *   mx_*        MXFP4 outputs as in fp4q_mxfp4_quant (mx_deq, mx_loss may be
+ *               NULL).
+ * cols % 32 == 0.  Errors as the separate calls; d_status collects both.
+ */
+fp4q_status fp4q_quantize_dual(const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                               const float* importance, const uint32_t* sign_masks, float* d_amax,
+                               uint8_t* nv_codes, uint8_t* nv_scales, float* d_global_scale,
+                               void* nv_deq, float* nv_loss, uint8_t* mx_codes, uint8_t* mx_scales,
+                               void* mx_deq, float* mx_loss, int32_t* d_status, fp4q_stream_t stream);
+
+/*
  * fp4q_dequant -- decode codes and scales back to values.
  * NVFP4: out = RN(q * RN(E4M3(s) * S)), S = *d_global_scale; MXFP4:
  * out = q * 2^(b-127); then rounded to `out_dt`.  Reproduces the `deq` output
