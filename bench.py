@@ -151,21 +151,60 @@ class Model:
             self.events = [(torch.cuda.Event(enable_timing=True, external=True),
                             torch.cuda.Event(enable_timing=True, external=True)) for _ in self.shapes]
         self.launches_per_step = 2 * len(self.shapes)
+        self.ready = [torch.cuda.Event() for _ in self.shapes]
+        self.done = [torch.cuda.Event() for _ in self.shapes]
 
-    def step(self, stream):
+    def step_schedule(self, streams, lag):
+        """MXFP4 passes on streams[0]; NVFP4 sweeps round-robin on streams[1:], each
+        after its own tensor's MXFP4 pass; with lag > 0 the MXFP4 pass of tensor t
+        also waits for the sweep of tensor t - lag to finish (keeps the two kinds of
+        kernels interleaved instead of letting the MXFP4 passes run ahead)."""
+        fq = self.fq
+        s0 = streams[0]
+        for s in streams[1:]:
+            s.wait_stream(s0)
+        for i, (w, o) in enumerate(zip(self.w, self.out)):
+            if lag > 0 and i >= lag:
+                s0.wait_event(self.done[i - lag])
+            fq.fp4q_mxfp4_quant_absmax(w, None, o["mx_codes"], o["mx_scales"], o["amax"], o["mx_deq"],
+                                       None, self.status, s0)
+            self.ready[i].record(s0)
+            s2 = streams[1 + i % (len(streams) - 1)]
+            s2.wait_event(self.ready[i])
+            if self.events is not None:
+                self.events[i][0].record(s2)
+            fq.fp4q_nvfp4_sweepmse(w, o["amax"], o["nv_codes"], o["nv_scales"], o["S"], o["nv_deq"],
+                                   None, self.status, s2)
+            if self.events is not None:
+                self.events[i][1].record(s2)
+            self.done[i].record(s2)
+        for s in streams[1:]:
+            s0.wait_stream(s)
+
+    def step(self, stream, stream2=None):
         """Per tensor: MXFP4 (which also reduces max|w|), then the NVFP4 ScaleSweep on
         that max -- the two launches of fp4q_quantize_dual, issued as its two C calls
-        so that events can bracket the NVFP4 sweep."""
+        so that events can bracket the NVFP4 sweep.  With `stream2` the sweeps run on
+        a second stream, each after its own tensor's MXFP4 pass, so that the sweep of
+        one tensor overlaps the MXFP4 pass of the next."""
         fq = self.fq
+        s2 = stream if stream2 is None else stream2
+        if stream2 is not None:
+            stream2.wait_stream(stream)
         for i, (w, o) in enumerate(zip(self.w, self.out)):
             fq.fp4q_mxfp4_quant_absmax(w, None, o["mx_codes"], o["mx_scales"], o["amax"], o["mx_deq"],
                                        None, self.status, stream)
+            if stream2 is not None:
+                self.ready[i].record(stream)
+                stream2.wait_event(self.ready[i])
             if self.events is not None:
-                self.events[i][0].record(stream)
+                self.events[i][0].record(s2)
             fq.fp4q_nvfp4_sweepmse(w, o["amax"], o["nv_codes"], o["nv_scales"], o["S"], o["nv_deq"],
-                                   None, self.status, stream)
+                                   None, self.status, s2)
             if self.events is not None:
-                self.events[i][1].record(stream)
+                self.events[i][1].record(s2)
+        if stream2 is not None:
+            stream.wait_stream(stream2)
 
     def sweep_ms(self):
         return [a.elapsed_time(b) for a, b in self.events]
@@ -374,6 +413,11 @@ def main():
     ap.add_argument("--single", choices=sorted(SINGLE_PATHS), default=None,
                     help="time one kernel on one tensor instead of the benchmark step")
     ap.add_argument("--shape", default="16384x8192")
+    ap.add_argument("--streams", type=int, default=2, choices=[1, 2, 3, 4],
+                    help="1: one stream; n > 1: MXFP4 passes on one stream, NVFP4 sweeps "
+                         "round-robin on n - 1 more, each after its own tensor's MXFP4 pass")
+    ap.add_argument("--lag", type=int, default=0,
+                    help="with --streams > 1: the MXFP4 pass of tensor t waits for the sweep of t - lag")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -399,13 +443,21 @@ def main():
 
     model = Model(fq, dev, seed=5 + 1000 * rank, with_events=True)
     stream = torch.cuda.Stream(device=dev)
+    streams = [stream] + [torch.cuda.Stream(device=dev) for _ in range(args.streams - 1)]
     stream.wait_stream(torch.cuda.current_stream())
     graph = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        model.step(stream)                       # eager warm-up before capture
-        stream.synchronize()
-        with torch.cuda.graph(graph, stream=stream):
+
+    def run_step():
+        if args.streams == 1:
             model.step(stream)
+        else:
+            model.step_schedule(streams, args.lag)
+
+    with torch.cuda.stream(stream):
+        run_step()                               # eager warm-up before capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=stream):
+            run_step()
     for _ in range(max(args.warmup, 3) - 1):
         graph.replay()
     torch.cuda.synchronize()
@@ -476,7 +528,9 @@ def main():
     }
     if rank == 0:
         try:
-            e2e_dt, h2d, d2h = e2e_run(fq, model, max(1, args.e2e_steps), dev)
+            if args.e2e_steps < 1:
+                raise RuntimeError("skipped (--e2e-steps 0)")
+            e2e_dt, h2d, d2h = e2e_run(fq, model, args.e2e_steps, dev)
             line["e2e"] = {"value": 2.0 * n / e2e_dt / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_dt * 1e3}
         except Exception as e:   # report, do not hide
