@@ -47,6 +47,7 @@ B_MXFP4 = 2.0 + 0.5 + 1.0 / 32 + 2.0
 # r = x*inv, E2M1(r), y = q*d, e = x - y, e*e, L + e*e
 OPS_PER_ELEM_CAND = 6
 NVFP4_MSE_CANDIDATES = 11
+MXFP4_CANDIDATES = 3
 SM_FP32_LANES = 128
 
 
@@ -153,6 +154,31 @@ class Model:
         self.launches_per_step = 2 * len(self.shapes)
         self.ready = [torch.cuda.Event() for _ in self.shapes]
         self.done = [torch.cuda.Event() for _ in self.shapes]
+
+    def batch_setup(self, chunk):
+        """Descriptors of every weight for fp4q_quantize_batch, split into launches of at
+        most `chunk` weights (one workspace each) with events around each launch."""
+        fq = self.fq
+        self.chunks = []
+        for base in range(0, len(self.w), chunk):
+            items = []
+            for w, o in zip(self.w[base:base + chunk], self.out[base:base + chunk]):
+                items.append(dict(w=w, amax=o["amax"], global_scale=o["S"], nv_codes=o["nv_codes"],
+                                  nv_scales=o["nv_scales"], nv_deq=o["nv_deq"], mx_codes=o["mx_codes"],
+                                  mx_scales=o["mx_scales"], mx_deq=o["mx_deq"]))
+            ws = torch.empty(fq.fp4q_batch_workspace_bytes(), dtype=torch.uint8, device=self.dev)
+            n = sum(it["w"].numel() for it in items)
+            ev = (torch.cuda.Event(enable_timing=True, external=True),
+                  torch.cuda.Event(enable_timing=True, external=True))
+            self.chunks.append((items, ws, n, ev))
+        self.launches_per_step = len(self.chunks)
+
+    def step_batch(self, stream):
+        """The whole model in one persistent launch per chunk of weights."""
+        for items, ws, _, ev in self.chunks:
+            ev[0].record(stream)
+            self.fq.fp4q_quantize_batch(items, ws, self.status, stream)
+            ev[1].record(stream)
 
     def step_schedule(self, streams, lag):
         """MXFP4 passes on streams[0]; NVFP4 sweeps round-robin on streams[1:], each
@@ -416,6 +442,10 @@ def main():
     ap.add_argument("--streams", type=int, default=2, choices=[1, 2, 3, 4],
                     help="1: one stream; n > 1: MXFP4 passes on one stream, NVFP4 sweeps "
                          "round-robin on n - 1 more, each after its own tensor's MXFP4 pass")
+    ap.add_argument("--mode", default="calls", choices=["batch", "calls"],
+                    help="batch: fp4q_quantize_batch (one persistent launch per chunk of weights); "
+                         "calls: two launches per weight (fp4q_mxfp4_quant_absmax + the NVFP4 sweep)")
+    ap.add_argument("--chunk", type=int, default=128, help="weights per batch launch (at most 128)")
     ap.add_argument("--lag", type=int, default=0,
                     help="with --streams > 1: the MXFP4 pass of tensor t waits for the sweep of t - lag")
     args = ap.parse_args()
@@ -447,8 +477,13 @@ def main():
     stream.wait_stream(torch.cuda.current_stream())
     graph = torch.cuda.CUDAGraph()
 
+    if args.mode == "batch":
+        model.batch_setup(args.chunk)
+
     def run_step():
-        if args.streams == 1:
+        if args.mode == "batch":
+            model.step_batch(stream)
+        elif args.streams == 1:
             model.step(stream)
         else:
             model.step_schedule(streams, args.lag)
@@ -486,31 +521,44 @@ def main():
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
-    # the NVFP4 sweep kernel: per-launch durations of the last timed step
-    sweep_ms = model.sweep_ms()
     status = int(model.status.item())
 
     hbm_peak, peak_kind, sm_max = load_peaks()
     n = model.elements
     bytes_in = 2.0 * n * world
     value = bytes_in / (ms * 1e-3) / 1e9
-    sweep_total_ms = sum(sweep_ms)
-    sweep_bytes = B_NVFP4 * n
-    sweep_gbs = sweep_bytes / (sweep_total_ms * 1e-3) / 1e9
     clock_mhz = clk.get("sm_mhz") or sm_max
     alu_peak = 148 * SM_FP32_LANES * clock_mhz * 1e6 / 1e12          # Tlane-op/s
-    alu_achieved = OPS_PER_ELEM_CAND * NVFP4_MSE_CANDIDATES * n / (sweep_total_ms * 1e-3) / 1e12
-    hbm_frac = sweep_gbs / hbm_peak
+    if args.mode == "batch":
+        # the batch kernel: per-launch durations of the last timed step
+        kname = "batch_kernel (NVFP4-MSE + MXFP4, bf16)"
+        kern_ms = sum(ev[0].elapsed_time(ev[1]) for _, _, _, ev in model.chunks)
+        kern_bytes = (B_NVFP4 + B_MXFP4) * n
+        kern_ops = OPS_PER_ELEM_CAND * (NVFP4_MSE_CANDIDATES + MXFP4_CANDIDATES) * n
+        n_launch = len(model.chunks)
+    else:
+        # the NVFP4 sweep kernel: per-launch durations of the last timed step
+        kname = "nvfp4_sweep_kernel (MSE, bf16)"
+        kern_ms = sum(model.sweep_ms())
+        kern_bytes = B_NVFP4 * n
+        kern_ops = OPS_PER_ELEM_CAND * NVFP4_MSE_CANDIDATES * n
+        n_launch = len(model.shapes)
+    kern_gbs = kern_bytes / (kern_ms * 1e-3) / 1e9
+    alu_achieved = kern_ops / (kern_ms * 1e-3) / 1e12
+    hbm_frac = kern_gbs / hbm_peak
     alu_frac = alu_achieved / alu_peak
+    per_launch = {"launches_per_step": n_launch, "mean_launch_ms": kern_ms / n_launch,
+                  "algorithmic_bytes_per_launch": kern_bytes / n_launch}
     if alu_frac > hbm_frac:
         roof = {"bound": "alu", "achieved": alu_achieved, "peak": alu_peak, "unit": "Tlane-op/s",
-                "frac": alu_frac, "traffic": None, "kernel": "nvfp4_sweep_kernel (MSE, bf16)",
+                "frac": alu_frac, "traffic": None, "kernel": kname,
                 "peak_basis": f"148 SMs x 128 fp32 lanes x {clock_mhz:.0f} MHz median SM clock",
-                "hbm": {"achieved": sweep_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_frac,
-                        "peak_kind": peak_kind}}
+                "ops_basis": f"{OPS_PER_ELEM_CAND} fp32 operations per element and candidate of the definition",
+                "hbm": {"achieved": kern_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_frac,
+                        "peak_kind": peak_kind}, **per_launch}
     else:
-        roof = {"bound": "hbm", "achieved": sweep_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_frac,
-                "traffic": None, "kernel": "nvfp4_sweep_kernel (MSE, bf16)", "peak_kind": peak_kind}
+        roof = {"bound": "hbm", "achieved": kern_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_frac,
+                "traffic": None, "kernel": kname, "peak_kind": peak_kind, **per_launch}
     step_bytes = (B_NVFP4 + B_MXFP4) * n
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -518,7 +566,8 @@ def main():
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD, "tensors": len(model.shapes), "elements": n,
                    "input_bytes": 2 * n, "l2": "inputs 13.96 GB > 126 MB L2, no flush",
-                   "parallelism": f"replicas x{world} (weak)", "graph": "one CUDA graph per step"},
+                   "parallelism": f"replicas x{world} (weak)", "graph": "one CUDA graph per step",
+                   "mode": args.mode},
         "elements_per_s": n * world / (ms * 1e-3),
         "hbm_frac_step": step_bytes / (ms * 1e-3) / 1e9 / hbm_peak,
         "roofline": roof,

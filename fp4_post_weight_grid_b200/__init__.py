@@ -26,23 +26,37 @@ __all__ = [
     "fp4q_global_absmax", "fp4q_nvfp4_sweepmse", "fp4q_nvfp4_sweepwmse", "fp4q_mxfp4_quant",
     "fp4q_mxfp4_quant_hadamard", "fp4q_mxfp4_quant_absmax", "fp4q_quantize_dual", "fp4q_dequant",
     "fp4q_probe_e2m1", "fp4q_probe_e4m3",
+    "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "BatchTensor", "quantize_batch",
     "NVFP4Result", "MXFP4Result", "nvfp4_quantize", "mxfp4_quantize", "quantize_dual", "dequantize",
-    "FLAG_NONFINITE", "FLAG_RANGE",
+    "FLAG_NONFINITE", "FLAG_RANGE", "FLAG_TIMEOUT",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libfp4q.so")
 _lib = None
 
-OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_NONFINITE, ERR_CUDA, ERR_RANGE = range(8)
+OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_NONFINITE, ERR_CUDA, ERR_RANGE, ERR_ARG = range(9)
 F32, BF16 = 0, 1
 NVFP4, MXFP4 = 0, 1
-FLAG_NONFINITE, FLAG_RANGE = 1, 2
+FLAG_NONFINITE, FLAG_RANGE, FLAG_TIMEOUT = 1, 2, 4
+BATCH_MAX = 128
 NVFP4_BLOCK, MXFP4_BLOCK = 16, 32
 EXPORTS = ("fp4q_version", "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_global_absmax",
            "fp4q_nvfp4_sweepmse", "fp4q_nvfp4_sweepwmse", "fp4q_mxfp4_quant",
-           "fp4q_mxfp4_quant_hadamard", "fp4q_mxfp4_quant_absmax", "fp4q_quantize_dual", "fp4q_dequant",
+           "fp4q_mxfp4_quant_hadamard", "fp4q_mxfp4_quant_absmax", "fp4q_quantize_dual",
+           "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_dequant",
            "fp4q_probe_e2m1", "fp4q_probe_e4m3")
+
+
+class BatchTensor(ctypes.Structure):
+    """Mirror of fp4q_batch_tensor (include/fp4q.h)."""
+    _fields_ = [("w", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("importance", ctypes.c_void_p), ("sign_masks", ctypes.c_void_p),
+                ("amax", ctypes.c_void_p), ("global_scale", ctypes.c_void_p),
+                ("nv_codes", ctypes.c_void_p), ("nv_scales", ctypes.c_void_p),
+                ("nv_deq", ctypes.c_void_p), ("nv_loss", ctypes.c_void_p),
+                ("mx_codes", ctypes.c_void_p), ("mx_scales", ctypes.c_void_p),
+                ("mx_deq", ctypes.c_void_p), ("mx_loss", ctypes.c_void_p)]
 
 
 class Fp4qError(RuntimeError):
@@ -87,10 +101,13 @@ def load():
         "fp4q_probe_e2m1": [P, P, I64, P],
         "fp4q_probe_e4m3": [P, P, I64, P],
     }
+    sigs["fp4q_quantize_batch"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, ctypes.c_size_t, P, P]
     for name, args in sigs.items():
         fn = getattr(lib, name)
         fn.restype = I
         fn.argtypes = args
+    lib.fp4q_batch_workspace_bytes.restype = ctypes.c_size_t
+    lib.fp4q_batch_workspace_bytes.argtypes = []
     _lib = lib
     return lib
 
@@ -239,6 +256,48 @@ def fp4q_quantize_dual(w, importance, sign_masks, d_amax, nv_codes, nv_scales, d
                                      cp, sp, dp, lp, st, _stream(stream)), "fp4q_quantize_dual")
 
 
+def fp4q_batch_workspace_bytes() -> int:
+    return int(load().fp4q_batch_workspace_bytes())
+
+
+def fp4q_quantize_batch(items, workspace: torch.Tensor, d_status: torch.Tensor, stream=None) -> None:
+    """Quantize a list of weights to NVFP4 and MXFP4 in one persistent launch per
+    BATCH_MAX weights.  `items` is a list of dicts with the fields of
+    fp4q_batch_tensor as CUDA tensors (w, amax, global_scale, nv_codes, nv_scales,
+    mx_codes, mx_scales required; importance, sign_masks, nv_deq, nv_loss, mx_deq,
+    mx_loss optional).  All weights share one dtype."""
+    if not items:
+        return
+    dt = _wdtype(items[0]["w"])
+    dev = items[0]["w"].device
+    arr = (BatchTensor * len(items))()
+    for k, it in enumerate(items):
+        w = it["w"]
+        if w.dtype != items[0]["w"].dtype:
+            raise TypeError("all weights of a batch share one dtype")
+        rows, cols = _rc(w, MXFP4_BLOCK)
+        n = rows * cols
+        arr[k].w = _dev(w, "w", device=dev)
+        arr[k].rows, arr[k].cols = rows, cols
+        arr[k].importance = _dev(it.get("importance"), "importance", torch.float32, cols, dev)
+        arr[k].sign_masks = _dev(it.get("sign_masks"), "sign_masks", (torch.int32, torch.uint32),
+                                 cols // MXFP4_BLOCK, dev)
+        arr[k].amax = _dev(it["amax"], "amax", torch.float32, 1, dev)
+        arr[k].global_scale = _dev(it["global_scale"], "global_scale", torch.float32, 1, dev)
+        arr[k].nv_codes = _dev(it["nv_codes"], "nv_codes", torch.uint8, n // 2, dev)
+        arr[k].nv_scales = _dev(it["nv_scales"], "nv_scales", torch.uint8, n // NVFP4_BLOCK, dev)
+        arr[k].nv_deq = _dev(it.get("nv_deq"), "nv_deq", w.dtype, n, dev)
+        arr[k].nv_loss = _dev(it.get("nv_loss"), "nv_loss", torch.float32, n // NVFP4_BLOCK, dev)
+        arr[k].mx_codes = _dev(it["mx_codes"], "mx_codes", torch.uint8, n // 2, dev)
+        arr[k].mx_scales = _dev(it["mx_scales"], "mx_scales", torch.uint8, n // MXFP4_BLOCK, dev)
+        arr[k].mx_deq = _dev(it.get("mx_deq"), "mx_deq", w.dtype, n, dev)
+        arr[k].mx_loss = _dev(it.get("mx_loss"), "mx_loss", torch.float32, n // MXFP4_BLOCK, dev)
+    wp = _dev(workspace, "workspace", torch.uint8, None, dev)
+    sp = _dev(d_status, "d_status", torch.int32, 1, dev)
+    _check(load().fp4q_quantize_batch(arr, len(items), dt, wp, workspace.numel(), sp, _stream(stream)),
+           "fp4q_quantize_batch")
+
+
 def fp4q_dequant(fmt: int, codes, scales, d_global_scale, rows: int, cols: int, out,
                  stream=None) -> None:
     """Decode codes + scales (+ S for NVFP4) into `out` (bf16 or fp32)."""
@@ -348,6 +407,41 @@ def quantize_dual(w: torch.Tensor, importance: Optional[torch.Tensor] = None,
     fp4q_quantize_dual(w, importance, sign_masks, amax, nv.codes, nv.scales, S, nv.deq, nv.block_loss,
                        mx.codes, mx.scales, mx.deq, mx.block_loss, status, stream)
     return nv, mx
+
+
+def quantize_batch(weights, importances=None, sign_masks=None, with_deq=True, with_loss=True,
+                   stream=None):
+    """NVFP4 and MXFP4 of every weight in `weights` (one dtype), in one launch per
+    BATCH_MAX weights; returns a list of (NVFP4Result, MXFP4Result) sharing one
+    status word."""
+    if not weights:
+        return []
+    dev = weights[0].device
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = torch.empty(fp4q_batch_workspace_bytes(), dtype=torch.uint8, device=dev)
+    items, out = [], []
+    for k, w in enumerate(weights):
+        rows, cols = _rc(w, MXFP4_BLOCK)
+        amax = torch.empty(1, dtype=torch.float32, device=dev)
+        S = torch.empty(1, dtype=torch.float32, device=dev)
+        nv = NVFP4Result(torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+                         torch.empty((rows, cols // NVFP4_BLOCK), dtype=torch.uint8, device=dev), S,
+                         torch.empty_like(w) if with_deq else None,
+                         torch.empty((rows, cols // NVFP4_BLOCK), dtype=torch.float32, device=dev)
+                         if with_loss else None, amax, status)
+        mx = MXFP4Result(torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+                         torch.empty((rows, cols // MXFP4_BLOCK), dtype=torch.uint8, device=dev),
+                         torch.empty_like(w) if with_deq else None,
+                         torch.empty((rows, cols // MXFP4_BLOCK), dtype=torch.float32, device=dev)
+                         if with_loss else None, status)
+        items.append(dict(w=w, importance=None if importances is None else importances[k],
+                          sign_masks=None if sign_masks is None else sign_masks[k], amax=amax,
+                          global_scale=S, nv_codes=nv.codes, nv_scales=nv.scales, nv_deq=nv.deq,
+                          nv_loss=nv.block_loss, mx_codes=mx.codes, mx_scales=mx.scales,
+                          mx_deq=mx.deq, mx_loss=mx.block_loss))
+        out.append((nv, mx))
+    fp4q_quantize_batch(items, ws, status, stream)
+    return out
 
 
 def dequantize(fmt: int, codes: torch.Tensor, scales: torch.Tensor, global_scale=None,

@@ -8,6 +8,7 @@
 
 #include <cuda_runtime.h>
 
+#include "batch.h"
 #include "fp4q.h"
 #include "launch.h"
 
@@ -104,6 +105,7 @@ const char* fp4q_status_string(fp4q_status status)
     case FP4Q_ERR_NONFINITE: return "non-finite input";
     case FP4Q_ERR_CUDA: return "CUDA launch error";
     case FP4Q_ERR_RANGE: return "max|x| outside the supported range";
+    case FP4Q_ERR_ARG: return "invalid argument (workspace too small)";
     }
     return "unknown status";
 }
@@ -232,6 +234,70 @@ fp4q_status fp4q_quantize_dual(const void* w, fp4q_dtype dt, int64_t rows, int64
     if (st != FP4Q_OK) return st;
     return nvfp4_common(w, dt, rows, cols, d_amax, importance, importance != nullptr, nv_codes, nv_scales,
                         d_global_scale, nv_deq, nv_loss, d_status, stream);
+}
+
+size_t fp4q_batch_workspace_bytes(void) { return (size_t)fp4q::kWsWords * sizeof(unsigned); }
+
+fp4q_status fp4q_quantize_batch(const fp4q_batch_tensor* tensors, int32_t n, fp4q_dtype dt,
+                                void* workspace, size_t workspace_bytes, int32_t* d_status,
+                                fp4q_stream_t stream)
+{
+    if (!valid_dtype(dt)) return FP4Q_ERR_DTYPE;
+    if (n < 0) return FP4Q_ERR_SHAPE;
+    if (n == 0) return FP4Q_OK;
+    if (!tensors || !workspace || !d_status) return FP4Q_ERR_NULL;
+    if (!aligned(workspace, 16) || !aligned(d_status, 4)) return FP4Q_ERR_ALIGN;
+    if (workspace_bytes < fp4q_batch_workspace_bytes()) return FP4Q_ERR_ARG;
+    for (int32_t i = 0; i < n; ++i) {          // check every descriptor before enqueueing
+        const fp4q_batch_tensor& t = tensors[i];
+        bool empty = false;
+        fp4q_status st = check_quant_args(t.w, dt, t.rows, t.cols, FP4Q_MXFP4_BLOCK, t.nv_codes, t.nv_scales,
+                                          d_status, t.nv_deq, t.nv_loss, 8, &empty);
+        if (st != FP4Q_OK) return st;
+        if (!empty) {
+            st = check_quant_args(t.w, dt, t.rows, t.cols, FP4Q_MXFP4_BLOCK, t.mx_codes, t.mx_scales,
+                                  d_status, t.mx_deq, t.mx_loss, 16, &empty);
+            if (st != FP4Q_OK) return st;
+        }
+        if (!t.amax || !t.global_scale) return FP4Q_ERR_NULL;
+        if (!aligned(t.amax, 4) || !aligned(t.global_scale, 4) ||
+            (t.importance && !aligned(t.importance, 16)) || (t.sign_masks && !aligned(t.sign_masks, 4)))
+            return FP4Q_ERR_ALIGN;
+    }
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    static thread_local fp4q::BatchParams p;     // ~19 KB: kept off the stack
+    for (int32_t base = 0; base < n; base += fp4q::kMaxBatch) {
+        const int32_t m = n - base < fp4q::kMaxBatch ? n - base : fp4q::kMaxBatch;
+        std::memset(&p, 0, sizeof(p));
+        p.n = m;
+        int64_t item = 0;
+        int seg = 0;
+        auto add = [&](int t, bool nv) {
+            const fp4q_batch_tensor& d = tensors[base + t];
+            p.seg_start[seg] = (int32_t)item;
+            p.seg_tensor[seg] = (int16_t)t;
+            p.seg_nv[seg] = nv ? 1 : 0;
+            item += nv ? fp4q::batch_nv_tiles(d.rows, d.cols) : fp4q::batch_mx_tiles(d.rows, d.cols);
+            ++seg;
+        };
+        // MX(0) MX(1) NV(0) MX(2) NV(1) ... MX(m-1) NV(m-2) NV(m-1)
+        add(0, false);
+        for (int t = 1; t < m; ++t) {
+            add(t, false);
+            add(t - 1, true);
+        }
+        add(m - 1, true);
+        if (item > INT32_MAX - 1) return FP4Q_ERR_SHAPE;
+        p.seg_start[seg] = (int32_t)item;
+        for (int t = 0; t < m; ++t) {
+            p.t[t] = tensors[base + t];
+            p.mx_tiles[t] = (int32_t)fp4q::batch_mx_tiles(p.t[t].rows, p.t[t].cols);
+        }
+        fp4q::launch_batch(p, dt == FP4Q_BF16, static_cast<unsigned*>(workspace), d_status, s);
+        const fp4q_status st = after_launch();
+        if (st != FP4Q_OK) return st;
+    }
+    return FP4Q_OK;
 }
 
 fp4q_status fp4q_dequant(fp4q_format format, const uint8_t* codes, const uint8_t* scales,

@@ -230,5 +230,6 @@ __device__ __forceinline__ void store_block(float* p, const float (&y)[N])
 
 constexpr int32_t kFlagNonfinite = 1;
 constexpr int32_t kFlagRange = 2;
+constexpr int32_t kFlagTimeout = 4;
 
 }  // namespace fp4q

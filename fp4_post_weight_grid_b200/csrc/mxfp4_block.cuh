@@ -1,0 +1,204 @@
+// mxfp4_block.cuh -- MXFP4 quantization of one 32-element block with the
+// E8M0 exponent sweep, optionally after the random-sign block Hadamard; shared
+// by the per-tensor kernel and the batch kernel.
+//
+// "Bridging the Gap Between Promise and Performance for Microscaling FP4
+// Quantization" (gist.science, arXiv 2509.23202), technical summary:
+//   sec. 1  MXFP4 groups of 32 elements share one power-of-two (E8M0) scale;
+//   sec. 2  the group scales are chosen to minimise the MSE ("Grade Otimizada
+//           por MSE"), and block Hadamard micro-rotations are fused into the
+//           GPU kernel ("Rotacoes Online Fundidas").
+// "Resumo Tecnico: TORQ" (arXiv 2605.19561) sec. 2.B: the S-step maps the
+// block maximum onto the largest code, which gives the centre exponent e0 =
+// the smallest e with 6*2^e >= amax; the sweep visits e0-1, e0, e0+1.
+//
+// One thread owns one block: the rotation (sign flips, five in-register
+// butterfly stages h = 1..16, the 1/sqrt(32) multiply) and the sequential loss
+// stay in registers.  The three exponents are selected by screen-then-verify
+// (screen.cuh) in units of 2^e0: e0-1 and e0 screened as a pair element by
+// element, e0+1 two elements at a time.  The Hadamard runs on the CUDA cores:
+// it has to reproduce the stage order bit for bit, which a tensor-core
+// contraction does not, and it costs 6 adds/multiplies per element against a
+// memory budget of ~4.5 bytes per element.
+#pragma once
+
+#include "device.cuh"
+#include "screen.cuh"
+
+namespace fp4q {
+
+constexpr float kInvSqrt32 = 0x1.6a09e6p-3f;   // RN(1/sqrt(32))
+
+// Quantize one 32-element block; returns max|w| (as binary32 bits) of the
+// unrotated block, for a fused global max.
+//   src      the block's 32 input elements; sign_mask: its sign mask (HAD only)
+//   codes16  16 bytes of packed nibbles; scale: the E8M0 byte
+//   deq32    32 reconstructed elements or nullptr; loss: the block's loss or nullptr
+template <typename T, bool HAD>
+__device__ __forceinline__ uint32_t mxfp4_block(const T* __restrict__ src, uint32_t sign_mask,
+                                                uint8_t* __restrict__ codes16, uint8_t* __restrict__ scale,
+                                                T* __restrict__ deq32, float* __restrict__ loss,
+                                                int32_t* __restrict__ d_status, uint64_t z2, float neg_zero)
+{
+    float x[32];
+    load_block<32>(src, x);
+    uint32_t wmax = 0;     // max |w| bits of the unrotated block
+    if (HAD) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) wmax = max(wmax, __float_as_uint(x[j]) & 0x7FFFFFFFu);
+    }
+    if (HAD) {
+        const uint32_t m = sign_mask;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            x[j] = __uint_as_float(__float_as_uint(x[j]) ^ (((m >> j) & 1u) << 31));
+#pragma unroll
+        for (int h = 1; h < 32; h *= 2) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (i & h) continue;
+                const float a = x[i], c = x[i + h];
+                x[i] = __fadd_rn(a, c);
+                x[i + h] = __fsub_rn(a, c);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = __fmul_rn(x[j], kInvSqrt32);
+    }
+    float a[32];        // |y|, shared by every stage below
+    uint32_t abits = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        a[j] = fabsf(x[j]);
+        abits = max(abits, __float_as_uint(a[j]));
+    }
+    if (abits >= 0x7F800000u) atomicOr(d_status, kFlagNonfinite);
+    if (!HAD) wmax = abits;
+    int e0 = -127;
+    if (abits >= 0x00800000u) {
+        const int a = (int)(abits >> 23) - 127;                 // floor(log2 amax)
+        e0 = a - 2 + ((abits & 0x7FFFFFu) > 0x400000u ? 1 : 0);  // 6*2^(a-2) = 1.5*2^a
+        e0 = min(max(e0, -127), 127);
+    }
+    // candidate k = 0, 1, 2 is the exponent e0 - 1 + k, clamped to [-127, 127]
+#define FP4Q_EK(k) min(max(e0 - 1 + (k), -127), 127)
+
+    // 1. screen the three exponents in units of 2^e0 (S = 2^e0, v = 2^(e-e0))
+    const float inv0 = exp2i(-e0);
+    float alpha2;
+    {
+        uint64_t al2 = pk(0.0f, 0.0f);
+        const uint64_t inv02 = pk(inv0, inv0);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const uint64_t as = mul2(pk(a[2 * j], a[2 * j + 1]), inv02);
+            al2 = fma2(as, as, al2);
+        }
+        float lo, hi;
+        upk(al2, lo, hi);
+        alpha2 = (lo + hi) * (1.0f + 0x1p-16f);   // bound only: rounded up generously
+    }
+    const float tS = 0x1p-70f * inv0;
+    const float tau = tS * tS + 0x1p-120f;
+    float lam[3];
+    {   // exponents e0-1 and e0 as a pair, one element at a time
+        const int ea = FP4Q_EK(0), eb = FP4Q_EK(1);
+        const uint64_t inv2 = pk(exp2i(-ea), exp2i(-eb));
+        uint64_t L2 = pk(0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            float ra, rb;
+            upk(mul2(pk(a[i], a[i]), inv2), ra, rb);
+            const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
+            L2 = fma2(et, et, L2);
+        }
+        upk(mul2(L2, pk(exp2i(2 * (ea - e0)), exp2i(2 * (eb - e0)))), lam[0], lam[1]);
+    }
+    {   // exponent e0+1, two elements at a time
+        const int ec = FP4Q_EK(2);
+        const float invc = exp2i(-ec);
+        const uint64_t inv2 = pk(invc, invc);
+        uint64_t L2 = pk(0.0f, 0.0f);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float ra, rb;
+            upk(mul2(pk(a[2 * j], a[2 * j + 1]), inv2), ra, rb);
+            const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
+            L2 = fma2(et, et, L2);
+        }
+        float lo, hi;
+        upk(L2, lo, hi);
+        lam[2] = (lo + hi) * exp2i(2 * (ec - e0));
+    }
+    const float M = fminf(fminf(lam[0], lam[1]), lam[2]);
+    const float thr = survivor_threshold(M, alpha2, tau);
+    uint32_t mask = (lam[0] <= thr ? 1u : 0u) | (lam[1] <= thr ? 2u : 0u) | (lam[2] <= thr ? 4u : 0u);
+    if (mask == 0) mask = 7u;                  // unreachable for finite inputs; evaluate all
+
+    // 2. verify: exact loss of the survivors, first minimum wins
+    int be;
+    if ((mask & (mask - 1)) == 0) {
+        be = FP4Q_EK(__ffs(mask) - 1);
+    } else {
+        float best = 0.0f;
+        bool first = true;
+        be = FP4Q_EK(0);
+        while (mask) {
+            const int k = __ffs(mask) - 1;
+            mask &= mask - 1;
+            const int e = FP4Q_EK(k);
+            const uint64_t d2 = pk(exp2i(e), exp2i(e)), inv2 = pk(exp2i(-e), exp2i(-e));
+            float L = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const uint64_t ap = pk(a[2 * j], a[2 * j + 1]);
+                float r0, r1;
+                upk(mul2(ap, inv2), r0, r1);
+                const uint64_t q2 = h2_to_f2(e2m1x2_round_h(r0, r1), neg_zero);
+                const uint64_t e2 = sub2(ap, mul2_nofuse(q2, d2, z2));
+                float s0, s1;
+                upk(mul2_nofuse(e2, e2, z2), s0, s1);
+                L = __fadd_rn(__fadd_rn(L, s0), s1);
+            }
+            if (first || L < best) { best = L; be = e; }
+            first = false;
+        }
+    }
+
+    // 3. emit the winner with its exact loss
+    const float d = exp2i(be), inv = exp2i(-be);
+    const uint64_t d2 = pk(d, d), inv2 = pk(inv, inv);
+    uint32_t word[4];
+    float L = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {          // 8 elements per chunk: one 16-byte bf16 store
+        float y[8];
+        word[c] = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = 8 * c + 2 * j;
+            const uint64_t xp = pk(x[i], x[i + 1]);
+            float r0, r1;
+            upk(mul2(xp, inv2), r0, r1);
+            const uint32_t byte = e2m1x2(r0, r1);
+            word[c] |= byte << (8 * j);
+            const uint64_t y2 = mul2_nofuse(h2_to_f2(e2m1x2_to_f16x2(byte), neg_zero), d2, z2);
+            upk(y2, y[2 * j], y[2 * j + 1]);
+            if (loss) {     // the winner is known; its exact loss is only an output
+                const uint64_t e2 = sub2(xp, y2);
+                float s0, s1;
+                upk(mul2_nofuse(e2, e2, z2), s0, s1);
+                L = __fadd_rn(__fadd_rn(L, s0), s1);
+            }
+        }
+        if (deq32) store_block<8>(deq32 + 8 * c, y);
+    }
+#undef FP4Q_EK
+    st_stream(codes16, make_uint4(word[0], word[1], word[2], word[3]));
+    *scale = (uint8_t)(be + 127);
+    if (loss) *loss = L;
+    return wmax;
+
+}
+
+}  // namespace fp4q

@@ -62,6 +62,7 @@
 #ifndef FP4Q_H
 #define FP4Q_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -79,7 +80,8 @@ typedef enum {
     FP4Q_ERR_ALIGN = 4,
     FP4Q_ERR_NONFINITE = 5,
     FP4Q_ERR_CUDA = 6,
-    FP4Q_ERR_RANGE = 7
+    FP4Q_ERR_RANGE = 7,
+    FP4Q_ERR_ARG = 8
 } fp4q_status;
 
 typedef enum { FP4Q_F32 = 0, FP4Q_BF16 = 1 } fp4q_dtype;
@@ -88,6 +90,7 @@ typedef enum { FP4Q_NVFP4 = 0, FP4Q_MXFP4 = 1 } fp4q_format;
 /* Bits OR-ed into *d_status by the device. */
 #define FP4Q_FLAG_NONFINITE 1  /* a NaN or Inf reached the scale search     */
 #define FP4Q_FLAG_RANGE     2  /* NVFP4: max|x| nonzero and outside [2^-64, 2^64] */
+#define FP4Q_FLAG_TIMEOUT   4  /* batch: a tile gave up waiting for its weight's max */
 
 #define FP4Q_NVFP4_BLOCK 16
 #define FP4Q_MXFP4_BLOCK 32
@@ -229,6 +232,63 @@ fp4q_status fp4q_quantize_dual(const void* w, fp4q_dtype dt, int64_t rows, int64
                                uint8_t* nv_codes, uint8_t* nv_scales, float* d_global_scale,
                                void* nv_deq, float* nv_loss, uint8_t* mx_codes, uint8_t* mx_scales,
                                void* mx_deq, float* mx_loss, int32_t* d_status, fp4q_stream_t stream);
+
+/*
+ * fp4q_quantize_batch -- fp4q_quantize_dual for a list of weights, in one
+ * persistent launch per FP4Q_BATCH_MAX weights.
+ * Thread blocks take 16384-element tiles from a device queue ordered
+ * MXFP4(0) MXFP4(1) NVFP4(0) MXFP4(2) NVFP4(1) ...: the MXFP4 tiles of a weight
+ * also reduce its max|w|, and its NVFP4 tiles (ScaleSweep summary,
+ * "Metodologia: ScaleSweep" secs. 2-3: S = max|x|/(256*6)) start once all of
+ * them have finished, so memory-bound and arithmetic-bound tiles share the
+ * SMs.  Results are identical to the single-weight calls.
+ *   tensors   HOST array of n descriptors; it is read during the call only
+ *             (the descriptors travel to the device as a kernel argument).
+ *             Per weight: w (16-byte aligned, rows x cols, cols % 32 == 0);
+ *             importance (NULL: NVFP4 MSE, else WMSE weights [cols]);
+ *             sign_masks (NULL: plain MXFP4, else the block Hadamard masks
+ *             [cols/32]); amax and global_scale (device floats, written);
+ *             nv_codes, nv_scales, nv_deq, nv_loss and mx_codes, mx_scales,
+ *             mx_deq, mx_loss as in fp4q_quantize_dual (deq/loss may be NULL).
+ *   dt        dtype of every w (and of every deq).
+ *   workspace device scratch of at least fp4q_batch_workspace_bytes()
+ *             bytes, 16-byte aligned, owned by the caller; zeroed by the call
+ *             (stream-ordered) before each launch.  Launches that overlap on
+ *             the device must not share a workspace.
+ *   d_status  FP4Q_FLAG_NONFINITE / FP4Q_FLAG_RANGE as the single calls, and
+ *             FP4Q_FLAG_TIMEOUT if an NVFP4 tile waited about two seconds for
+ *             its weight's MXFP4 tiles (the tile is then skipped; this does
+ *             not happen when the tiles make progress).
+ * An empty weight (rows or cols == 0) gets amax = 0 and global_scale = 1.
+ * Errors: FP4Q_ERR_SHAPE (n < 0, a bad shape), FP4Q_ERR_NULL, FP4Q_ERR_ALIGN,
+ * FP4Q_ERR_DTYPE, FP4Q_ERR_ARG (workspace too small), FP4Q_ERR_CUDA; the
+ * descriptors are all checked before anything is enqueued.
+ */
+#define FP4Q_BATCH_MAX 128
+
+typedef struct {
+    const void* w;
+    int64_t rows;
+    int64_t cols;
+    const float* importance;
+    const uint32_t* sign_masks;
+    float* amax;
+    float* global_scale;
+    uint8_t* nv_codes;
+    uint8_t* nv_scales;
+    void* nv_deq;
+    float* nv_loss;
+    uint8_t* mx_codes;
+    uint8_t* mx_scales;
+    void* mx_deq;
+    float* mx_loss;
+} fp4q_batch_tensor;
+
+size_t fp4q_batch_workspace_bytes(void);
+
+fp4q_status fp4q_quantize_batch(const fp4q_batch_tensor* tensors, int32_t n, fp4q_dtype dt,
+                                void* workspace, size_t workspace_bytes, int32_t* d_status,
+                                fp4q_stream_t stream);
 
 /*
  * fp4q_dequant -- decode codes and scales back to values.

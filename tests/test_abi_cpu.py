@@ -78,6 +78,38 @@ def test_argument_errors_without_a_gpu(fq):
     assert lib.fp4q_dequant(1, None, None, None, 0, 32, None, 0, None) == fq.OK
 
 
+def test_batch_argument_errors_without_a_gpu(fq):
+    lib = fq.load()
+    buf = ctypes.create_string_buffer(4096)
+    p = ctypes.addressof(buf)
+    p16 = p + (-p % 16)
+    ws = fq.fp4q_batch_workspace_bytes()
+    assert ws >= 4 * (4 + 2 * fq.BATCH_MAX)
+
+    def one(**kw):
+        t = fq.BatchTensor()
+        for f, _ in fq.BatchTensor._fields_:
+            setattr(t, f, p16)
+        t.rows, t.cols, t.importance, t.sign_masks = 2, 64, None, None
+        t.nv_deq = t.nv_loss = t.mx_deq = t.mx_loss = None
+        for k, v in kw.items():
+            setattr(t, k, v)
+        arr = (fq.BatchTensor * 1)(t)
+        return lib.fp4q_quantize_batch(arr, 1, 1, p16, ws, p16, None)
+
+    assert one(cols=48) == fq.ERR_SHAPE
+    assert one(rows=-1) == fq.ERR_SHAPE
+    assert one(w=None) == fq.ERR_NULL
+    assert one(amax=None) == fq.ERR_NULL
+    assert one(w=p16 + 2) == fq.ERR_ALIGN
+    assert one(mx_codes=p16 + 8) == fq.ERR_ALIGN
+    arr = (fq.BatchTensor * 1)()
+    assert lib.fp4q_quantize_batch(arr, 1, 1, p16, ws - 1, p16, None) == fq.ERR_ARG
+    assert lib.fp4q_quantize_batch(arr, 1, 9, p16, ws, p16, None) == fq.ERR_DTYPE
+    assert lib.fp4q_quantize_batch(arr, -1, 1, p16, ws, p16, None) == fq.ERR_SHAPE
+    assert lib.fp4q_quantize_batch(arr, 0, 1, None, 0, None, None) == fq.OK
+
+
 def test_binding_refuses_cpu_tensors(fq):
     w = torch.zeros((4, 32), dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
