@@ -26,7 +26,8 @@ __all__ = [
     "fp4q_global_absmax", "fp4q_nvfp4_sweepmse", "fp4q_nvfp4_sweepwmse", "fp4q_mxfp4_quant",
     "fp4q_mxfp4_quant_hadamard", "fp4q_mxfp4_quant_absmax", "fp4q_quantize_dual", "fp4q_dequant",
     "fp4q_probe_e2m1", "fp4q_probe_e4m3",
-    "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "BatchTensor", "quantize_batch",
+    "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_quantize_batch_static", "BatchTensor",
+    "quantize_batch",
     "NVFP4Result", "MXFP4Result", "nvfp4_quantize", "mxfp4_quantize", "quantize_dual", "dequantize",
     "FLAG_NONFINITE", "FLAG_RANGE", "FLAG_TIMEOUT",
 ]
@@ -44,7 +45,7 @@ NVFP4_BLOCK, MXFP4_BLOCK = 16, 32
 EXPORTS = ("fp4q_version", "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_global_absmax",
            "fp4q_nvfp4_sweepmse", "fp4q_nvfp4_sweepwmse", "fp4q_mxfp4_quant",
            "fp4q_mxfp4_quant_hadamard", "fp4q_mxfp4_quant_absmax", "fp4q_quantize_dual",
-           "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_dequant",
+           "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_quantize_batch_static", "fp4q_dequant",
            "fp4q_probe_e2m1", "fp4q_probe_e4m3")
 
 
@@ -102,6 +103,7 @@ def load():
         "fp4q_probe_e4m3": [P, P, I64, P],
     }
     sigs["fp4q_quantize_batch"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, ctypes.c_size_t, P, P]
+    sigs["fp4q_quantize_batch_static"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, P]
     for name, args in sigs.items():
         fn = getattr(lib, name)
         fn.restype = I
@@ -258,6 +260,47 @@ def fp4q_quantize_dual(w, importance, sign_masks, d_amax, nv_codes, nv_scales, d
 
 def fp4q_batch_workspace_bytes() -> int:
     return int(load().fp4q_batch_workspace_bytes())
+
+
+def _batch_array(items):
+    """fp4q_batch_tensor array of the descriptor dicts (argument marshalling)."""
+    dev = items[0]["w"].device
+    arr = (BatchTensor * len(items))()
+    for k, it in enumerate(items):
+        w = it["w"]
+        if w.dtype != items[0]["w"].dtype:
+            raise TypeError("all weights of a batch share one dtype")
+        rows, cols = _rc(w, MXFP4_BLOCK)
+        n = rows * cols
+        arr[k].w = _dev(w, "w", device=dev)
+        arr[k].rows, arr[k].cols = rows, cols
+        arr[k].importance = _dev(it.get("importance"), "importance", torch.float32, cols, dev)
+        arr[k].sign_masks = _dev(it.get("sign_masks"), "sign_masks", (torch.int32, torch.uint32),
+                                 cols // MXFP4_BLOCK, dev)
+        arr[k].amax = _dev(it["amax"], "amax", torch.float32, 1, dev)
+        arr[k].global_scale = _dev(it["global_scale"], "global_scale", torch.float32, 1, dev)
+        arr[k].nv_codes = _dev(it["nv_codes"], "nv_codes", torch.uint8, n // 2, dev)
+        arr[k].nv_scales = _dev(it["nv_scales"], "nv_scales", torch.uint8, n // NVFP4_BLOCK, dev)
+        arr[k].nv_deq = _dev(it.get("nv_deq"), "nv_deq", w.dtype, n, dev)
+        arr[k].nv_loss = _dev(it.get("nv_loss"), "nv_loss", torch.float32, n // NVFP4_BLOCK, dev)
+        arr[k].mx_codes = _dev(it["mx_codes"], "mx_codes", torch.uint8, n // 2, dev)
+        arr[k].mx_scales = _dev(it["mx_scales"], "mx_scales", torch.uint8, n // MXFP4_BLOCK, dev)
+        arr[k].mx_deq = _dev(it.get("mx_deq"), "mx_deq", w.dtype, n, dev)
+        arr[k].mx_loss = _dev(it.get("mx_loss"), "mx_loss", torch.float32, n // MXFP4_BLOCK, dev)
+    return arr, dev
+
+
+def fp4q_quantize_batch_static(items, d_status: torch.Tensor, stream=None) -> None:
+    """fp4q_quantize_batch with the library's own static scratch instead of a
+    caller-provided workspace (at most BATCH_MAX weights; allocates nothing)."""
+    if len(items) > BATCH_MAX:
+        raise Fp4qError(ERR_ARG, f"fp4q_quantize_batch_static takes at most {BATCH_MAX} weights")
+    if not items:
+        return
+    arr, dev = _batch_array(items)
+    sp = _dev(d_status, "d_status", torch.int32, 1, dev)
+    _check(load().fp4q_quantize_batch_static(arr, len(items), _wdtype(items[0]["w"]), sp, _stream(stream)),
+           "fp4q_quantize_batch_static")
 
 
 def fp4q_quantize_batch(items, workspace: torch.Tensor, d_status: torch.Tensor, stream=None) -> None:

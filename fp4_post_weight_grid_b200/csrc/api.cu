@@ -300,6 +300,22 @@ fp4q_status fp4q_quantize_batch(const fp4q_batch_tensor* tensors, int32_t n, fp4
     return FP4Q_OK;
 }
 
+fp4q_status fp4q_quantize_batch_static(const fp4q_batch_tensor* tensors, int32_t n, fp4q_dtype dt,
+                                       int32_t* d_status, fp4q_stream_t stream)
+{
+    if (n > FP4Q_BATCH_MAX) return FP4Q_ERR_ARG;    // the static scratch serves one launch
+    if (n <= 0) return fp4q_quantize_batch(tensors, n, dt, nullptr, 0, d_status, stream);
+    unsigned* ws = nullptr;
+    size_t bytes = 0;
+    const cudaError_t e = fp4q::batch_static_workspace(&ws, &bytes);
+    if (e != cudaSuccess) {
+        std::strncpy(g_last_cuda_error, cudaGetErrorString(e), sizeof(g_last_cuda_error) - 1);
+        g_last_cuda_error[sizeof(g_last_cuda_error) - 1] = '\0';
+        return FP4Q_ERR_CUDA;
+    }
+    return fp4q_quantize_batch(tensors, n, dt, ws, bytes, d_status, stream);
+}
+
 fp4q_status fp4q_dequant(fp4q_format format, const uint8_t* codes, const uint8_t* scales,
                          const float* d_global_scale, int64_t rows, int64_t cols, void* out,
                          fp4q_dtype out_dt, fp4q_stream_t stream)

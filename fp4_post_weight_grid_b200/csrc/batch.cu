@@ -18,6 +18,8 @@
 //
 // The per-block arithmetic is exactly that of the single-weight kernels
 // (nvfp4_block.cuh, mxfp4_block.cuh), so the results are bit-identical.
+#include <mutex>
+
 #include "batch.h"
 #include "device.cuh"
 #include "launch.h"
@@ -159,6 +161,33 @@ batch_kernel(const __grid_constant__ BatchParams P, unsigned* __restrict__ ws, i
 }
 
 }  // namespace
+
+// Scratch of fp4q_quantize_batch_static: the tile queue counter and the
+// per-weight max and completion counters of one launch (kWsWords words).  It
+// lives in the library's own device memory, so every GPU that loads the
+// library holds it until the process exits; host code only ever sees a
+// stand-in for it and gets its device address from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned g_static_ws[kWsWords];
+
+cudaError_t batch_static_workspace(unsigned** ws, size_t* bytes)
+{
+    static std::mutex mu;
+    static unsigned* addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {                       // once per device, with that device current
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_ws);
+        if (e != cudaSuccess) return e;
+        addr[dev] = static_cast<unsigned*>(p);
+    }
+    *ws = addr[dev];
+    *bytes = sizeof(g_static_ws);
+    return cudaSuccess;
+}
 
 int64_t batch_mx_tiles(int64_t rows, int64_t cols)
 {

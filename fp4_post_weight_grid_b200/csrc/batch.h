@@ -28,4 +28,8 @@ int64_t batch_mx_tiles(int64_t rows, int64_t cols);
 int64_t batch_nv_tiles(int64_t rows, int64_t cols);
 void launch_batch(const BatchParams& p, bool bf16, unsigned* ws, int32_t* d_status, cudaStream_t s);
 
+// Device address and size of the library's own batch scratch (batch.cu); the
+// first call on a device looks the address up.
+cudaError_t batch_static_workspace(unsigned** ws, size_t* bytes);
+
 }  // namespace fp4q

@@ -291,6 +291,31 @@ fp4q_status fp4q_quantize_batch(const fp4q_batch_tensor* tensors, int32_t n, fp4
                                 fp4q_stream_t stream);
 
 /*
+ * fp4q_quantize_batch_static -- fp4q_quantize_batch without a caller-provided
+ * workspace, for callers that cannot allocate device memory when they
+ * quantize: a process whose device memory is handed out entirely by another
+ * allocator (so that an extra cudaMalloc could fail or fragment its pool), a
+ * fixed device-memory budget set at start-up, or a latency-critical path that
+ * must not call cudaMalloc (which can synchronize the device).  The pages have
+ * no counterpart; this is a library convenience.
+ * The scratch (the tile queue counter and the per-weight max and completion
+ * counters, a little over 1 KB) is a static array inside the library, which
+ * every GPU that loads the library holds until the process exits.  The call
+ * allocates nothing and calls no allocating routine.
+ *   n         at most FP4Q_BATCH_MAX weights per call (one launch); more
+ *             returns FP4Q_ERR_ARG before anything is enqueued.
+ * Other arguments, results and errors as fp4q_quantize_batch.
+ * The first call on a device looks up the scratch's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  The scratch is zeroed, stream-ordered, at the
+ * start of every call, but it is shared by all calls on a device: calls whose
+ * launches overlap on the GPU (different streams without ordering between
+ * them) race on it and give wrong results.
+ */
+fp4q_status fp4q_quantize_batch_static(const fp4q_batch_tensor* tensors, int32_t n, fp4q_dtype dt,
+                                       int32_t* d_status, fp4q_stream_t stream);
+
+/*
  * fp4q_dequant -- decode codes and scales back to values.
  * NVFP4: out = RN(q * RN(E4M3(s) * S)), S = *d_global_scale; MXFP4:
  * out = q * 2^(b-127); then rounded to `out_dt`.  Reproduces the `deq` output
