@@ -41,7 +41,7 @@ __device__ __forceinline__ unsigned ld_volatile(const unsigned* p)
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 4)
 batch_kernel(const __grid_constant__ BatchParams P, unsigned* __restrict__ ws, int32_t* __restrict__ d_status,
              float neg_zero)
 {

@@ -86,6 +86,27 @@ __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte)
     return r;
 }
 
+// Four pairs r[2j], r[2j+1] (j = 0..3) -> one word of four code bytes (pair j
+// in byte j, r[2j] in its low nibble), and the four decoded pairs as f16x2.
+// The code bytes stay in 8-bit PTX registers between the conversions.
+__device__ __forceinline__ uint32_t e2m1x8_encode(const float (&r)[8], uint32_t (&h2)[4])
+{
+    uint32_t w;
+    asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t0, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t1, %8, %7;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t2, %10, %9;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t3, %12, %11;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, t0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, t1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, t2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %4, t3;\n\t"
+        "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
+        : "=r"(w), "=r"(h2[0]), "=r"(h2[1]), "=r"(h2[2]), "=r"(h2[3])
+        : "f"(r[0]), "f"(r[1]), "f"(r[2]), "f"(r[3]), "f"(r[4]), "f"(r[5]), "f"(r[6]), "f"(r[7]));
+    return w;
+}
+
 // f16x2 -> two binary32 (exact).
 __device__ __forceinline__ void f16x2_to_f32(uint32_t h2, float& lo, float& hi)
 {
@@ -94,6 +115,14 @@ __device__ __forceinline__ void f16x2_to_f32(uint32_t h2, float& lo, float& hi)
         "cvt.f32.f16 %0, a;\n\t"
         "cvt.f32.f16 %1, b;\n\t}"
         : "=f"(lo), "=f"(hi) : "r"(h2));
+}
+
+// f16x2 -> binary32 pair (exact).
+__device__ __forceinline__ uint64_t f16x2_to_f2(uint32_t h2)
+{
+    float lo, hi;
+    f16x2_to_f32(h2, lo, hi);
+    return pk(lo, hi);
 }
 
 // Decoded E2M1 value pair of one code byte, as binary32.
@@ -201,6 +230,40 @@ __device__ __forceinline__ void load_block(const float* p, float (&x)[N])
         x[4 * v + 2] = __uint_as_float(u.z);
         x[4 * v + 3] = __uint_as_float(u.w);
     }
+}
+
+// load_block that also returns max |x| as binary32 bits (NaN above Inf above
+// every finite value).  bf16: the maximum is taken on the raw 16-bit halves.
+template <int N>
+__device__ __forceinline__ void load_block_amax(const __nv_bfloat16* p, float (&x)[N], uint32_t& amax_bits)
+{
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int v = 0; v < N / 8; ++v) {
+        uint4 u = ld_stream(p + 8 * v);
+        bf16x2_to_f32(u.x, x[8 * v + 0], x[8 * v + 1]);
+        bf16x2_to_f32(u.y, x[8 * v + 2], x[8 * v + 3]);
+        bf16x2_to_f32(u.z, x[8 * v + 4], x[8 * v + 5]);
+        bf16x2_to_f32(u.w, x[8 * v + 6], x[8 * v + 7]);
+        m2 = __vmaxu2(m2, __vmaxu2(u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu));
+        m2 = __vmaxu2(m2, __vmaxu2(u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu));
+    }
+    amax_bits = max(m2 & 0xFFFFu, m2 >> 16) << 16;
+}
+template <int N>
+__device__ __forceinline__ void load_block_amax(const float* p, float (&x)[N], uint32_t& amax_bits)
+{
+    uint32_t m = 0;
+#pragma unroll
+    for (int v = 0; v < N / 4; ++v) {
+        uint4 u = ld_stream(p + 4 * v);
+        x[4 * v + 0] = __uint_as_float(u.x);
+        x[4 * v + 1] = __uint_as_float(u.y);
+        x[4 * v + 2] = __uint_as_float(u.z);
+        x[4 * v + 3] = __uint_as_float(u.w);
+        m = max(m, max(max(u.x & 0x7FFFFFFFu, u.y & 0x7FFFFFFFu), max(u.z & 0x7FFFFFFFu, u.w & 0x7FFFFFFFu)));
+    }
+    amax_bits = m;
 }
 
 // Store N binary32 values rounded to the element type.

@@ -14,7 +14,7 @@ constexpr int kThreads = 256;
 // max on the binary32 bit pattern, which keeps NaN and Inf), for the NVFP4
 // global scale of the same weight.
 template <typename T, bool HAD, bool AMAX>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 4)
 mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
              const uint32_t* __restrict__ masks, uint8_t* __restrict__ codes,
              uint8_t* __restrict__ scales, T* __restrict__ deq, float* __restrict__ loss,

@@ -15,8 +15,7 @@
 // One thread owns one block: the rotation (sign flips, five in-register
 // butterfly stages h = 1..16, the 1/sqrt(32) multiply) and the sequential loss
 // stay in registers.  The three exponents are selected by screen-then-verify
-// (screen.cuh) in units of 2^e0: e0-1 and e0 screened as a pair element by
-// element, e0+1 two elements at a time.  The Hadamard runs on the CUDA cores:
+// (screen.cuh) in units of 2^e0, each exponent two elements at a time.  The Hadamard runs on the CUDA cores:
 // it has to reproduce the stage order bit for bit, which a tensor-core
 // contraction does not, and it costs 6 adds/multiplies per element against a
 // memory budget of ~4.5 bytes per element.
@@ -41,12 +40,9 @@ __device__ __forceinline__ uint32_t mxfp4_block(const T* __restrict__ src, uint3
                                                 int32_t* __restrict__ d_status, uint64_t z2, float neg_zero)
 {
     float x[32];
-    load_block<32>(src, x);
-    uint32_t wmax = 0;     // max |w| bits of the unrotated block
-    if (HAD) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) wmax = max(wmax, __float_as_uint(x[j]) & 0x7FFFFFFFu);
-    }
+    uint32_t wmax;         // max |w| bits of the unrotated block
+    load_block_amax<32>(src, x, wmax);
+    uint32_t abits = wmax; // max |y| bits of the block that is quantized
     if (HAD) {
         const uint32_t m = sign_mask;
 #pragma unroll
@@ -64,16 +60,13 @@ __device__ __forceinline__ uint32_t mxfp4_block(const T* __restrict__ src, uint3
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[j] = __fmul_rn(x[j], kInvSqrt32);
-    }
-    float a[32];        // |y|, shared by every stage below
-    uint32_t abits = 0;
+        abits = 0;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        a[j] = fabsf(x[j]);
-        abits = max(abits, __float_as_uint(a[j]));
+        for (int j = 0; j < 32; ++j) abits = max(abits, __float_as_uint(x[j]) & 0x7FFFFFFFu);
     }
+    // From here on the search works on the signed values: E2M1 rounding and
+    // every loss term are symmetric in the sign.
     if (abits >= 0x7F800000u) atomicOr(d_status, kFlagNonfinite);
-    if (!HAD) wmax = abits;
     int e0 = -127;
     if (abits >= 0x00800000u) {
         const int a = (int)(abits >> 23) - 127;                 // floor(log2 amax)
@@ -85,50 +78,36 @@ __device__ __forceinline__ uint32_t mxfp4_block(const T* __restrict__ src, uint3
 
     // 1. screen the three exponents in units of 2^e0 (S = 2^e0, v = 2^(e-e0))
     const float inv0 = exp2i(-e0);
-    float alpha2;
-    {
-        uint64_t al2 = pk(0.0f, 0.0f);
-        const uint64_t inv02 = pk(inv0, inv0);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const uint64_t as = mul2(pk(a[2 * j], a[2 * j + 1]), inv02);
-            al2 = fma2(as, as, al2);
-        }
-        float lo, hi;
-        upk(al2, lo, hi);
-        alpha2 = (lo + hi) * (1.0f + 0x1p-16f);   // bound only: rounded up generously
-    }
+    const float as = __uint_as_float(abits) * inv0;      // sum y^2 / S^2 <= 32 amax^2 / S^2
+    const float alpha2 = (32.0f * as * as) * (1.0f + 0x1p-16f);
     const float tS = 0x1p-70f * inv0;
     const float tau = tS * tS + 0x1p-120f;
     float lam[3];
-    {   // exponents e0-1 and e0 as a pair, one element at a time
-        const int ea = FP4Q_EK(0), eb = FP4Q_EK(1);
-        const uint64_t inv2 = pk(exp2i(-ea), exp2i(-eb));
-        uint64_t L2 = pk(0.0f, 0.0f);
+    {   // the three exponents, two elements at a time
+        uint64_t inv2[3], L2[3];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            float ra, rb;
-            upk(mul2(pk(a[i], a[i]), inv2), ra, rb);
-            const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
-            L2 = fma2(et, et, L2);
+        for (int k = 0; k < 3; ++k) {
+            const float ik = exp2i(-FP4Q_EK(k));
+            inv2[k] = pk(ik, ik);
+            L2[k] = pk(0.0f, 0.0f);
         }
-        upk(mul2(L2, pk(exp2i(2 * (ea - e0)), exp2i(2 * (eb - e0)))), lam[0], lam[1]);
-    }
-    {   // exponent e0+1, two elements at a time
-        const int ec = FP4Q_EK(2);
-        const float invc = exp2i(-ec);
-        const uint64_t inv2 = pk(invc, invc);
-        uint64_t L2 = pk(0.0f, 0.0f);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            float ra, rb;
-            upk(mul2(pk(a[2 * j], a[2 * j + 1]), inv2), ra, rb);
-            const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
-            L2 = fma2(et, et, L2);
+            const uint64_t xp = pk(x[2 * j], x[2 * j + 1]);
+#pragma unroll
+            for (int k = 0; k < 3; ++k) {
+                float ra, rb;
+                upk(mul2(xp, inv2[k]), ra, rb);
+                const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
+                L2[k] = fma2(et, et, L2[k]);
+            }
         }
-        float lo, hi;
-        upk(L2, lo, hi);
-        lam[2] = (lo + hi) * exp2i(2 * (ec - e0));
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            float lo, hi;
+            upk(L2[k], lo, hi);
+            lam[k] = (lo + hi) * exp2i(2 * (FP4Q_EK(k) - e0));
+        }
     }
     const float M = fminf(fminf(lam[0], lam[1]), lam[2]);
     const float thr = survivor_threshold(M, alpha2, tau);
@@ -151,11 +130,11 @@ __device__ __forceinline__ uint32_t mxfp4_block(const T* __restrict__ src, uint3
             float L = 0.0f;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const uint64_t ap = pk(a[2 * j], a[2 * j + 1]);
+                const uint64_t xp = pk(x[2 * j], x[2 * j + 1]);
                 float r0, r1;
-                upk(mul2(ap, inv2), r0, r1);
+                upk(mul2(xp, inv2), r0, r1);
                 const uint64_t q2 = h2_to_f2(e2m1x2_round_h(r0, r1), neg_zero);
-                const uint64_t e2 = sub2(ap, mul2_nofuse(q2, d2, z2));
+                const uint64_t e2 = sub2(xp, mul2_nofuse(q2, d2, z2));
                 float s0, s1;
                 upk(mul2_nofuse(e2, e2, z2), s0, s1);
                 L = __fadd_rn(__fadd_rn(L, s0), s1);
@@ -172,20 +151,18 @@ __device__ __forceinline__ uint32_t mxfp4_block(const T* __restrict__ src, uint3
     float L = 0.0f;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {          // 8 elements per chunk: one 16-byte bf16 store
-        float y[8];
-        word[c] = 0;
+        float y[8], r[8];
+        uint32_t q2[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) upk(mul2(pk(x[8 * c + 2 * j], x[8 * c + 2 * j + 1]), inv2), r[2 * j], r[2 * j + 1]);
+        word[c] = e2m1x8_encode(r, q2);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int i = 8 * c + 2 * j;
-            const uint64_t xp = pk(x[i], x[i + 1]);
-            float r0, r1;
-            upk(mul2(xp, inv2), r0, r1);
-            const uint32_t byte = e2m1x2(r0, r1);
-            word[c] |= byte << (8 * j);
-            const uint64_t y2 = mul2_nofuse(h2_to_f2(e2m1x2_to_f16x2(byte), neg_zero), d2, z2);
+            const uint64_t y2 = mul2_nofuse(f16x2_to_f2(q2[j]), d2, z2);
             upk(y2, y[2 * j], y[2 * j + 1]);
             if (loss) {     // the winner is known; its exact loss is only an output
-                const uint64_t e2 = sub2(xp, y2);
+                const uint64_t e2 = sub2(pk(x[i], x[i + 1]), y2);
                 float s0, s1;
                 upk(mul2_nofuse(e2, e2, z2), s0, s1);
                 L = __fadd_rn(__fadd_rn(L, s0), s1);

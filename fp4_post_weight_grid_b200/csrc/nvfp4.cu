@@ -13,7 +13,7 @@ namespace {
 constexpr int kThreads = 256;
 
 template <typename T, int LO, int NREAL, bool WMSE>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, WMSE ? 3 : 5)
 nvfp4_sweep_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
                    const float* __restrict__ d_amax, const float* __restrict__ importance,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,

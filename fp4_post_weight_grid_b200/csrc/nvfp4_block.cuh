@@ -14,7 +14,7 @@
 // sequentially in column order in one thread's registers.  The candidate is
 // selected by screen-then-verify (screen.cuh): every candidate of the window
 // is screened in step units (two candidates per packed operation, element by
-// element so that the (|x|, |x|) pair is built once; an odd last candidate two
+// element so that the (x, x) pair is built once; an odd last candidate two
 // elements at a time), candidates whose screened loss exceeds the rigorous
 // threshold are dropped, the rest are evaluated with the exact definition,
 // and the emit stage writes the winner's codes, its reconstruction q*d and,
@@ -97,9 +97,13 @@ __device__ __forceinline__ void nvfp4_block(const NvTables& tb, const NvScale& c
                                             float* __restrict__ loss, uint64_t z2, float neg_zero)
 {
     constexpr int NC = (NREAL + 1) & ~1;
+    // The search works on the signed values: E2M1 rounding and every loss
+    // term are symmetric in the sign, so the losses equal those of |x|.
     float x[16];
-    load_block<16>(src, x);
-    float amax = 0.0f, alpha2 = 0.0f;
+    uint32_t abits;
+    load_block_amax<16>(src, x, abits);
+    const float amax = __uint_as_float(abits);
+    float alpha2;
     float wt[16];
     float tau = c.tau0;
     bool prune = true;
@@ -116,22 +120,19 @@ __device__ __forceinline__ void nvfp4_block(const NvTables& tb, const NvScale& c
         // the bound assumes 0 <= w <= 2^64 (sign bit clear, at most 2^64)
         prune = wbits <= 0x5F800000u;
         tau = c.tau0 * (1.0f + __uint_as_float(min(wbits, 0x5F800000u)));
-    }
-    float a[16];        // |x|, shared by every stage below
+        uint64_t al2 = pk(0.0f, 0.0f);
+        const uint64_t invS2 = pk(c.invS, c.invS);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) a[i] = fabsf(x[i]);
-    uint64_t al2 = pk(0.0f, 0.0f);
-    const uint64_t invS2 = pk(c.invS, c.invS);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        amax = fmaxf(amax, fmaxf(a[2 * j], a[2 * j + 1]));
-        const uint64_t as = mul2(pk(a[2 * j], a[2 * j + 1]), invS2);
-        al2 = fma2(WMSE ? mul2(pk(wt[2 * j], wt[2 * j + 1]), as) : as, as, al2);
-    }
-    {
+        for (int j = 0; j < 8; ++j) {
+            const uint64_t xs = mul2(pk(x[2 * j], x[2 * j + 1]), invS2);
+            al2 = fma2(mul2(pk(wt[2 * j], wt[2 * j + 1]), xs), xs, al2);
+        }
         float lo, hi;
         upk(al2, lo, hi);
         alpha2 = (lo + hi) * (1.0f + 0x1p-16f);   // bound only: rounded up generously
+    } else {
+        const float as = amax * c.invS;            // sum x^2 / S^2 <= 16 amax^2 / S^2
+        alpha2 = (16.0f * as * as) * (1.0f + 0x1p-16f);
     }
     const int p = (int)e4m3_rn_sat(__fdiv_rn(amax, c.t6));   // s_base pattern
 
@@ -147,8 +148,8 @@ __device__ __forceinline__ void nvfp4_block(const NvTables& tb, const NvScale& c
             L2[k] = pk(0.0f, 0.0f);
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {     // element outer: the (|x|, |x|) pair is built once
-            const uint64_t aa = pk(a[i], a[i]);
+        for (int i = 0; i < 16; ++i) {     // element outer: the (x, x) pair is built once
+            const uint64_t aa = pk(x[i], x[i]);
             const uint64_t w2 = WMSE ? pk(wt[i], wt[i]) : 0;
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
@@ -170,7 +171,7 @@ __device__ __forceinline__ void nvfp4_block(const NvTables& tb, const NvScale& c
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             float ra, rb;
-            upk(mul2(pk(a[2 * j], a[2 * j + 1]), inv2), ra, rb);
+            upk(mul2(pk(x[2 * j], x[2 * j + 1]), inv2), ra, rb);
             const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
             L2 = fma2(WMSE ? mul2(pk(wt[2 * j], wt[2 * j + 1]), et) : et, et, L2);
         }
@@ -204,11 +205,11 @@ __device__ __forceinline__ void nvfp4_block(const NvTables& tb, const NvScale& c
             float L = 0.0f;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const uint64_t ap = pk(a[2 * j], a[2 * j + 1]);
+                const uint64_t xp = pk(x[2 * j], x[2 * j + 1]);
                 float r0, r1;
-                upk(mul2(ap, inv2), r0, r1);
+                upk(mul2(xp, inv2), r0, r1);
                 const uint64_t q2 = h2_to_f2(e2m1x2_round_h(r0, r1), neg_zero);
-                const uint64_t e2 = sub2(ap, mul2_nofuse(q2, d2, z2));
+                const uint64_t e2 = sub2(xp, mul2_nofuse(q2, d2, z2));
                 uint64_t s2 = mul2_nofuse(e2, e2, z2);
                 if (WMSE) s2 = mul2_nofuse(pk(wt[2 * j], wt[2 * j + 1]), s2, z2);
                 float s0, s1;
@@ -224,30 +225,32 @@ __device__ __forceinline__ void nvfp4_block(const NvTables& tb, const NvScale& c
     //    and its exact loss when requested
     const float4 sw = tb.step[bp];
     const uint64_t d2 = pk(sw.x, sw.x), inv2 = pk(sw.y, sw.y);
-    uint32_t byte[8];
+    uint32_t word[2];
     float y[16];
     float L = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint64_t xp = pk(x[2 * j], x[2 * j + 1]);
-        float r0, r1;
-        upk(mul2(xp, inv2), r0, r1);
-        byte[j] = e2m1x2(r0, r1);
-        const uint64_t y2 = mul2_nofuse(h2_to_f2(e2m1x2_to_f16x2(byte[j]), neg_zero), d2, z2);
-        upk(y2, y[2 * j], y[2 * j + 1]);
-        if (loss) {     // the winner is known; its exact loss is only an output
-            const uint64_t e2 = sub2(xp, y2);
-            uint64_t s2 = mul2_nofuse(e2, e2, z2);
-            if (WMSE) s2 = mul2_nofuse(pk(wt[2 * j], wt[2 * j + 1]), s2, z2);
-            float s0, s1;
-            upk(s2, s0, s1);
-            L = __fadd_rn(__fadd_rn(L, s0), s1);
+    for (int h = 0; h < 2; ++h) {
+        float r[8];
+        uint32_t q2[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) upk(mul2(pk(x[8 * h + 2 * j], x[8 * h + 2 * j + 1]), inv2), r[2 * j], r[2 * j + 1]);
+        word[h] = e2m1x8_encode(r, q2);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = 8 * h + 2 * j;
+            const uint64_t y2 = mul2_nofuse(f16x2_to_f2(q2[j]), d2, z2);
+            upk(y2, y[i], y[i + 1]);
+            if (loss) {     // the winner is known; its exact loss is only an output
+                const uint64_t e2 = sub2(pk(x[i], x[i + 1]), y2);
+                uint64_t s2 = mul2_nofuse(e2, e2, z2);
+                if (WMSE) s2 = mul2_nofuse(pk(wt[i], wt[i + 1]), s2, z2);
+                float s0, s1;
+                upk(s2, s0, s1);
+                L = __fadd_rn(__fadd_rn(L, s0), s1);
+            }
         }
     }
-    uint2 packed;
-    packed.x = byte[0] | byte[1] << 8 | byte[2] << 16 | byte[3] << 24;
-    packed.y = byte[4] | byte[5] << 8 | byte[6] << 16 | byte[7] << 24;
-    st_stream64(codes8, packed);
+    st_stream64(codes8, make_uint2(word[0], word[1]));
     *scale = (uint8_t)bp;
     if (loss) *loss = L;
     if (deq16) store_block<16>(deq16, y);

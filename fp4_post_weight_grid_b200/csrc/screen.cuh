@@ -32,10 +32,9 @@
 //    lam_k - D(lam_k) <= U; using sqrt(z) <= (z/sqrt(U) + sqrt(U))/2 this holds
 //    whenever lam_k <= T = (U + u*K2*alpha*sqrt(U)/2 + K3*u^2*alpha^2 + tau) /
 //    (1 - u*K1 - u*K2*alpha/(2*sqrt(U))), so every candidate with lam_k > T is
-//    excluded.  T is evaluated with approximate sqrt/divide and then widened
-//    by 2^-10 relative, far more than their errors.  When the denominator is
-//    small (a block reproduced almost exactly) T is infinite and nothing is
-//    excluded.
+//    excluded.  survivor_threshold evaluates an upper bound of T with
+//    approximate square roots and reciprocals, each widened, and widens the
+//    result by another 2^-10 relative, far more than their errors.
 // 3. Verify.  The survivors (the screening minimum always survives; on
 //    typical weights about 1.002 per block) are evaluated with the exact
 //    definition in ascending order and the first minimum wins.  With a single
@@ -55,37 +54,53 @@ constexpr float kK1 = 128.0f;
 constexpr float kK2 = 16.0f;
 constexpr float kK3 = 64.0f;
 
+// Approximate square root, reciprocal square root and reciprocal (flush-to-zero
+// forms, single hardware instructions); callers widen every result so that the
+// threshold only grows, and pass normal inputs.
 __device__ __forceinline__ float sqrt_approx(float x)
 {
     float r;
-    asm("sqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
     return r;
 }
 
-__device__ __forceinline__ float div_approx(float a, float b)
+__device__ __forceinline__ float rsqrt_approx(float x)
 {
     float r;
-    asm("div.approx.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
     return r;
 }
 
 // Largest screened loss that can still belong to the exact winner.
 //   M      minimum screened loss lam over the candidates
-//   alpha2 ||x||^2 / S^2 (or the weighted norm), already rounded up
-//   tau    absolute allowance, in units of S^2
+//   alpha2 an upper bound of ||x||^2 / S^2 (or of the weighted norm); the
+//          bound D grows with alpha, so any upper bound keeps it valid
+//   tau    absolute allowance, in units of S^2 (at least 2^-120)
+// With a = 1 - u*K1, b = u*K2*alpha and c >= M + K3*u^2*alpha^2 + tau:
+//   sqrt(U) = (b + sqrt(b^2 + 4*a*c')) / (2a) <= (b + sqrt(c)) / a =: s (c' <= c),
+// and 1/s <= min(rho, 1/b) with rho >= 1/sqrt(c).  Any t > 0 may stand for
+// sqrt(U) in the bound sqrt(z) <= (z/t + t)/2; with t = s,
+//   T = (s^2 + b*s/2 + K3*u^2*alpha^2 + tau) / (1 - u*K1 - min(b*rho/2, 1/2)),
+// whose denominator is at least 1/2 - u*K1 (every candidate is kept if a NaN
+// makes it fail the test below).
 __device__ __forceinline__ float survivor_threshold(float M, float alpha2, float tau)
 {
-    const float alpha = sqrt_approx(alpha2) * (1.0f + 0x1p-16f);
-    const float b = kU * kK2 * alpha;
-    const float k3 = kK3 * kU * kU * alpha2;
+    const float alpha = sqrt_approx(fmaxf(alpha2, 0x1p-126f)) * (1.0f + 0x1p-16f);
+    const float hb = (0.5f * kU * kK2) * alpha;                    // b/2
+    const float k3 = (kK3 * kU * kU) * alpha2;
     const float c = (M + k3 + tau) * (1.0f + 0x1p-16f);
-    const float a1 = 1.0f - kU * kK1;
-    const float disc = b * b + 4.0f * a1 * c;
-    const float s = div_approx(b + sqrt_approx(disc), 2.0f * a1) * (1.0f + 0x1p-16f);  // sqrt(U)
-    const float U = s * s;
-    const float den = 1.0f - kU * kK1 - div_approx(b, 2.0f * s);
-    if (!(den > 0.25f)) return __int_as_float(0x7F800000);                            // keep all
-    const float T = div_approx(U + 0.5f * b * s + k3 + tau, den);
+    const float rho = rsqrt_approx(c) * (1.0f + 0x1p-16f);         // >= 1/sqrt(c)
+    const float s = (2.0f * hb + c * rho) * (1.0f + 0x1p-15f);    // >= sqrt(U)
+    const float den = (1.0f - kU * kK1) - fminf(hb * rho, 0.5f);
+    if (!(den > 0.25f)) return __int_as_float(0x7F800000);          // keep all
+    const float T = (s * s + hb * s + k3 + tau) * rcp_approx(den);
     return T * (1.0f + 0x1p-10f);
 }
 
