@@ -349,6 +349,28 @@ def run_reference(args):
     return 0
 
 
+# --------------------------------------------------------------------------- measured DRAM traffic
+# dram__bytes_read.sum + dram__bytes_write.sum of one nvfp4_sweep_kernel (MSE, bf16)
+# launch on a 16384 x 8192 weight, per element, with the sources it was taken on
+# (profiles/nvfp4_sweep_mse_16384x8192.md).  Traffic grows in proportion to the
+# elements, so a launch of n elements moves about n times this.  Once the sources
+# differ the figure no longer describes the kernel and none is reported.
+NVFP4_TRAFFIC = {"bytes_per_element": 556360704 / (16384 * 8192),
+                 "sources": ("nvfp4.cu", "nvfp4_block.cuh", "screen.cuh", "device.cuh"),
+                 "sha256": "6bca92bddfc55825b97e6db03fd9f5ecf560acb991e9d7009fe272f1d38c7bb8"}
+
+
+def measured_traffic_per_launch(elements_per_launch):
+    import hashlib
+    h = hashlib.sha256()
+    for f in NVFP4_TRAFFIC["sources"]:
+        with open(os.path.join(ROOT, "fp4_post_weight_grid_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != NVFP4_TRAFFIC["sha256"]:
+        return None
+    return NVFP4_TRAFFIC["bytes_per_element"] * elements_per_launch
+
+
 # --------------------------------------------------------------------------- single-kernel mode
 
 SINGLE_PATHS = {
@@ -357,6 +379,7 @@ SINGLE_PATHS = {
     "nvfp4-mse": (B_NVFP4, "nvfp4_sweep_kernel MSE"),
     "nvfp4-wmse": (B_NVFP4, "nvfp4_sweep_kernel WMSE"),
     "mxfp4": (B_MXFP4, "mxfp4_kernel"),
+    "mxfp4-absmax": (B_MXFP4, "mxfp4_kernel with the fused global max"),
     "mxfp4-hadamard": (B_MXFP4, "mxfp4_kernel Hadamard"),
     "dequant-nvfp4": (0.5 + 1.0 / 16 + 2.0, "dequant_kernel NVFP4"),
 }
@@ -398,6 +421,8 @@ def run_single(args):
             fq.fp4q_nvfp4_sweepwmse(w, amax, imp, codes, sc16, S, deq, None, st, stream)
         elif args.single == "mxfp4":
             fq.fp4q_mxfp4_quant(w, codes, sc32, deq, None, st, stream)
+        elif args.single == "mxfp4-absmax":
+            fq.fp4q_mxfp4_quant_absmax(w, None, codes, sc32, amax, deq, None, st, stream)
         elif args.single == "mxfp4-hadamard":
             fq.fp4q_mxfp4_quant_hadamard(w, masks, codes, sc32, deq, None, st, stream)
         elif args.single == "dequant-nvfp4":
@@ -549,16 +574,19 @@ def main():
     alu_frac = alu_achieved / alu_peak
     per_launch = {"launches_per_step": n_launch, "mean_launch_ms": kern_ms / n_launch,
                   "algorithmic_bytes_per_launch": kern_bytes / n_launch}
+    traffic = None
+    if args.mode != "batch":
+        traffic = measured_traffic_per_launch(kern_bytes / n_launch / B_NVFP4)
     if alu_frac > hbm_frac:
         roof = {"bound": "alu", "achieved": alu_achieved, "peak": alu_peak, "unit": "Tlane-op/s",
-                "frac": alu_frac, "traffic": None, "kernel": kname,
+                "frac": alu_frac, "traffic": traffic, "kernel": kname,
                 "peak_basis": f"148 SMs x 128 fp32 lanes x {clock_mhz:.0f} MHz median SM clock",
                 "ops_basis": f"{OPS_PER_ELEM_CAND} fp32 operations per element and candidate of the definition",
                 "hbm": {"achieved": kern_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_frac,
                         "peak_kind": peak_kind}, **per_launch}
     else:
         roof = {"bound": "hbm", "achieved": kern_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_frac,
-                "traffic": None, "kernel": kname, "peak_kind": peak_kind, **per_launch}
+                "traffic": traffic, "kernel": kname, "peak_kind": peak_kind, **per_launch}
     step_bytes = (B_NVFP4 + B_MXFP4) * n
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
