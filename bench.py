@@ -451,6 +451,75 @@ def run_single(args):
     return 0
 
 
+# --------------------------------------------------------------------------- per-call latency
+
+ACT_SHAPES = [(1, 4096), (16, 4096), (128, 4096), (1, 14336), (16, 14336), (2048, 4096), (4096, 14336)]
+
+
+def run_act_latency(args):
+    """Per-call latency of the NVFP4 sweep of a tensor quantized per call (an
+    activation: tokens x hidden): the two-call path (fp4q_global_absmax, then
+    fp4q_nvfp4_sweepmse) against the one-launch fp4q_nvfp4_sweep_dynamic, each
+    issued `--steps` times back to back on one stream, eagerly and as one CUDA
+    graph holding all the calls (device time per call without host launch
+    cost); CUDA events around the whole run.  Prints one JSON line
+    per shape (not the benchmark line)."""
+    import fp4_post_weight_grid_b200 as fq
+    from fp4_post_weight_grid_b200 import build as fbuild
+    import synth
+    fbuild.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream()
+    reps = max(args.steps, 20)
+    for rows, cols in ACT_SHAPES:
+        x = synth.t_weight(rows, cols, nu=4, scale=0.02, seed=13, device=dev)
+        amax = torch.empty(1, device=dev)
+        S = torch.empty(1, device=dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+        deq = torch.empty_like(x)
+        ws = torch.zeros(fq.fp4q_dynamic_workspace_bytes() // 4, dtype=torch.int32, device=dev)
+
+        def two():
+            fq.fp4q_global_absmax(x, amax, stream)
+            fq.fp4q_nvfp4_sweepmse(x, amax, codes, scales, S, deq, None, st, stream)
+
+        def one():
+            fq.fp4q_nvfp4_sweep_dynamic(x, None, amax, codes, scales, S, deq, None, ws, st, stream)
+
+        res = {"act_latency": [rows, cols], "reps": reps}
+        for name, fn in (("two_calls", two), ("dynamic", one)):
+            for _ in range(max(args.warmup, 3)):
+                fn()
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            res[name + "_eager_us"] = a.elapsed_time(b) * 1e3 / reps
+            g = torch.cuda.CUDAGraph()                 # `reps` calls in one graph
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(reps):
+                    fn()
+            g.replay()
+            torch.cuda.synchronize()
+            a.record(stream)
+            with torch.cuda.stream(stream):
+                g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            res[name + "_graph_us"] = a.elapsed_time(b) * 1e3 / reps
+            del g
+        res["status"] = int(st.item())
+        print(json.dumps(res), flush=True)
+    return 0
+
+
 # --------------------------------------------------------------------------- main
 
 def main():
@@ -461,6 +530,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--act-latency", action="store_true",
+                    help="per-call latency of the NVFP4 sweep on activation-sized tensors, two calls vs one launch")
     ap.add_argument("--single", choices=sorted(SINGLE_PATHS), default=None,
                     help="time one kernel on one tensor instead of the benchmark step")
     ap.add_argument("--shape", default="16384x8192")
@@ -478,6 +549,8 @@ def main():
         return run_reference(args)
     if args.single:
         return run_single(args)
+    if args.act_latency:
+        return run_act_latency(args)
 
     import fp4_post_weight_grid_b200 as fq
     from fp4_post_weight_grid_b200 import build as fbuild

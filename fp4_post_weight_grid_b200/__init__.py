@@ -27,6 +27,7 @@ __all__ = [
     "fp4q_mxfp4_quant_hadamard", "fp4q_mxfp4_quant_absmax", "fp4q_quantize_dual", "fp4q_dequant",
     "fp4q_probe_e2m1", "fp4q_probe_e4m3",
     "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_quantize_batch_static", "BatchTensor",
+    "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes", "nvfp4_quantize_dynamic",
     "quantize_batch",
     "NVFP4Result", "MXFP4Result", "nvfp4_quantize", "mxfp4_quantize", "quantize_dual", "dequantize",
     "FLAG_NONFINITE", "FLAG_RANGE", "FLAG_TIMEOUT",
@@ -46,7 +47,7 @@ EXPORTS = ("fp4q_version", "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_g
            "fp4q_nvfp4_sweepmse", "fp4q_nvfp4_sweepwmse", "fp4q_mxfp4_quant",
            "fp4q_mxfp4_quant_hadamard", "fp4q_mxfp4_quant_absmax", "fp4q_quantize_dual",
            "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_quantize_batch_static", "fp4q_dequant",
-           "fp4q_probe_e2m1", "fp4q_probe_e4m3")
+           "fp4q_probe_e2m1", "fp4q_probe_e4m3", "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes")
 
 
 class BatchTensor(ctypes.Structure):
@@ -104,12 +105,15 @@ def load():
     }
     sigs["fp4q_quantize_batch"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, ctypes.c_size_t, P, P]
     sigs["fp4q_quantize_batch_static"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, P]
+    sigs["fp4q_nvfp4_sweep_dynamic"] = [P, I, I64, I64, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]
     for name, args in sigs.items():
         fn = getattr(lib, name)
         fn.restype = I
         fn.argtypes = args
     lib.fp4q_batch_workspace_bytes.restype = ctypes.c_size_t
     lib.fp4q_batch_workspace_bytes.argtypes = []
+    lib.fp4q_dynamic_workspace_bytes.restype = ctypes.c_size_t
+    lib.fp4q_dynamic_workspace_bytes.argtypes = []
     _lib = lib
     return lib
 
@@ -256,6 +260,24 @@ def fp4q_quantize_dual(w, importance, sign_masks, d_amax, nv_codes, nv_scales, d
     mp = _dev(sign_masks, "sign_masks", (torch.int32, torch.uint32), cols // MXFP4_BLOCK, w.device)
     _check(load().fp4q_quantize_dual(wp, _wdtype(w), rows, cols, ip, mp, ap, ncp, nsp, gp, ndp, nlp,
                                      cp, sp, dp, lp, st, _stream(stream)), "fp4q_quantize_dual")
+
+
+def fp4q_dynamic_workspace_bytes() -> int:
+    return int(load().fp4q_dynamic_workspace_bytes())
+
+
+def fp4q_nvfp4_sweep_dynamic(x, importance, d_amax, codes, scales, d_global_scale, deq, block_loss,
+                             workspace: torch.Tensor, d_status, stream=None) -> None:
+    """Global max and NVFP4 ScaleSweep (MSE, or WMSE with `importance`) in one
+    cooperative launch.  `workspace`: a zeroed CUDA tensor of at least
+    fp4q_dynamic_workspace_bytes() bytes, left zeroed by the call."""
+    rows, cols, xp, ap, cp, sp, gp, dp, lp, st = _nvfp4_args(x, d_amax, codes, scales,
+                                                            d_global_scale, deq, block_loss, d_status)
+    ip = _dev(importance, "importance", torch.float32, cols, x.device)
+    wsp = _dev(workspace, "workspace", device=x.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load().fp4q_nvfp4_sweep_dynamic(xp, _wdtype(x), rows, cols, ip, ap, cp, sp, gp, dp, lp, wsp, nbytes,
+                                           st, _stream(stream)), "fp4q_nvfp4_sweep_dynamic")
 
 
 def fp4q_batch_workspace_bytes() -> int:
@@ -407,6 +429,28 @@ def nvfp4_quantize(w: torch.Tensor, importance: Optional[torch.Tensor] = None, w
         fp4q_nvfp4_sweepmse(w, amax, codes, scales, S, deq, loss, status, stream)
     else:
         fp4q_nvfp4_sweepwmse(w, amax, importance, codes, scales, S, deq, loss, status, stream)
+    return NVFP4Result(codes, scales, S, deq, loss, amax, status)
+
+
+def nvfp4_quantize_dynamic(x: torch.Tensor, importance: Optional[torch.Tensor] = None,
+                           workspace: Optional[torch.Tensor] = None, with_deq=True, with_loss=True,
+                           stream=None) -> NVFP4Result:
+    """nvfp4_quantize in one launch (fp4q_nvfp4_sweep_dynamic).  Pass a zeroed
+    `workspace` to reuse it across calls on one stream; by default a fresh one
+    is allocated."""
+    rows, cols = _rc(x, NVFP4_BLOCK)
+    dev = x.device
+    kw = dict(device=dev)
+    amax = torch.empty(1, dtype=torch.float32, **kw)
+    S = torch.empty(1, dtype=torch.float32, **kw)
+    status = torch.zeros(1, dtype=torch.int32, **kw)
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, **kw)
+    scales = torch.empty((rows, cols // NVFP4_BLOCK), dtype=torch.uint8, **kw)
+    deq = torch.empty_like(x) if with_deq else None
+    loss = torch.empty((rows, cols // NVFP4_BLOCK), dtype=torch.float32, **kw) if with_loss else None
+    if workspace is None:
+        workspace = torch.zeros(fp4q_dynamic_workspace_bytes() // 4, dtype=torch.int32, **kw)
+    fp4q_nvfp4_sweep_dynamic(x, importance, amax, codes, scales, S, deq, loss, workspace, status, stream)
     return NVFP4Result(codes, scales, S, deq, loss, amax, status)
 
 

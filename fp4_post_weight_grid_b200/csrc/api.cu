@@ -236,6 +236,43 @@ fp4q_status fp4q_quantize_dual(const void* w, fp4q_dtype dt, int64_t rows, int64
                         d_global_scale, nv_deq, nv_loss, d_status, stream);
 }
 
+size_t fp4q_dynamic_workspace_bytes(void) { return 16; }
+
+fp4q_status fp4q_nvfp4_sweep_dynamic(const void* x, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                     const float* importance, float* d_amax, uint8_t* codes,
+                                     uint8_t* scales_e4m3, float* d_global_scale, void* deq,
+                                     float* block_loss, void* workspace, size_t workspace_bytes,
+                                     int32_t* d_status, fp4q_stream_t stream)
+{
+    if (!valid_dtype(dt)) return FP4Q_ERR_DTYPE;
+    if (!shape_ok(rows, cols, FP4Q_NVFP4_BLOCK)) return FP4Q_ERR_SHAPE;
+    if (!d_amax) return FP4Q_ERR_NULL;
+    if (!aligned(d_amax, 4)) return FP4Q_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (rows == 0 || cols == 0) {      // max over no elements: 0
+        cudaMemsetAsync(d_amax, 0, sizeof(float), s);
+        return after_launch();
+    }
+    bool empty = false;
+    fp4q_status st = check_quant_args(x, dt, rows, cols, FP4Q_NVFP4_BLOCK, codes, scales_e4m3, d_status,
+                                      deq, block_loss, 8, &empty);
+    if (st != FP4Q_OK) return st;
+    if (!d_global_scale || !workspace) return FP4Q_ERR_NULL;
+    if (!aligned(d_global_scale, 4) || !aligned(workspace, 16) || (importance && !aligned(importance, 16)))
+        return FP4Q_ERR_ALIGN;
+    if (workspace_bytes < fp4q_dynamic_workspace_bytes()) return FP4Q_ERR_ARG;
+    const cudaError_t e = fp4q::launch_nvfp4_dynamic(x, dt == FP4Q_BF16, rows, cols, importance, d_amax, codes,
+                                                     scales_e4m3, d_global_scale, deq, block_loss,
+                                                     static_cast<unsigned*>(workspace), d_status, s);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        std::strncpy(g_last_cuda_error, cudaGetErrorString(e), sizeof(g_last_cuda_error) - 1);
+        g_last_cuda_error[sizeof(g_last_cuda_error) - 1] = '\0';
+        return FP4Q_ERR_CUDA;
+    }
+    return after_launch();
+}
+
 size_t fp4q_batch_workspace_bytes(void) { return (size_t)fp4q::kWsWords * sizeof(unsigned); }
 
 fp4q_status fp4q_quantize_batch(const fp4q_batch_tensor* tensors, int32_t n, fp4q_dtype dt,

@@ -44,6 +44,11 @@ void launch_mxfp4(const void* w, bool bf16, int64_t rows, int64_t cols, const ui
                   uint8_t* codes, uint8_t* scales, void* deq, float* loss, int32_t* d_status,
                   float* d_amax, cudaStream_t s);
 
+// NVFP4 global max + ScaleSweep in one cooperative launch; ws: 3 zeroed words.
+cudaError_t launch_nvfp4_dynamic(const void* w, bool bf16, int64_t rows, int64_t cols, const float* importance,
+                                 float* d_amax, uint8_t* codes, uint8_t* scales, float* d_S, void* deq,
+                                 float* loss, unsigned* ws, int32_t* d_status, cudaStream_t s);
+
 void launch_dequant(bool mx, const uint8_t* codes, const uint8_t* scales, const float* d_S,
                     int64_t rows, int64_t cols, void* out, bool out_bf16, cudaStream_t s);
 

@@ -234,6 +234,48 @@ fp4q_status fp4q_quantize_dual(const void* w, fp4q_dtype dt, int64_t rows, int64
                                void* mx_deq, float* mx_loss, int32_t* d_status, fp4q_stream_t stream);
 
 /*
+ * fp4q_dynamic_workspace_bytes -- size of the workspace of
+ * fp4q_nvfp4_sweep_dynamic (16 bytes).
+ */
+size_t fp4q_dynamic_workspace_bytes(void);
+
+/*
+ * fp4q_nvfp4_sweep_dynamic -- fp4q_global_absmax followed by
+ * fp4q_nvfp4_sweepmse (importance == NULL) or fp4q_nvfp4_sweepwmse, in ONE
+ * launch, for tensors quantized at every call (the activations of the
+ * weights+activations configurations, ScaleSweep summary "Resultados
+ * Experimentais"; S = max|x|/(256*6), "Metodologia: ScaleSweep" sec. 2).
+ * The global max and the sweep are separated by a barrier inside the launch:
+ * tensors of at most 16 x 256 16-element blocks run as one thread-block
+ * cluster (hardware cluster barriers, maxima exchanged through distributed
+ * shared memory; the workspace is not touched), larger ones as a cooperative
+ * launch (every thread block resident at once) with a grid-wide barrier on
+ * the workspace.  The bytes written are those of the two separate calls.
+ *   x, dt, rows, cols        as fp4q_nvfp4_sweepmse (cols % 16 == 0).
+ *   importance               device or NULL (cols floats, 16-byte aligned).
+ *   d_amax, d_global_scale   device floats, written (max|x| and S).
+ *   codes, scales_e4m3, deq, block_loss   as fp4q_nvfp4_sweepmse.
+ *   workspace                device, 16-byte aligned, at least
+ *                            fp4q_dynamic_workspace_bytes() bytes, ZEROED
+ *                            before its first use.  Every call leaves it
+ *                            zeroed again, except one that raised
+ *                            FP4Q_FLAG_TIMEOUT (zero it again after that).
+ *                            Calls that may run at the same time need
+ *                            separate workspaces.
+ * The barrier wait is bounded (about two seconds); on expiry
+ * FP4Q_FLAG_TIMEOUT is raised and the sweep is skipped.  Errors otherwise as
+ * the separate calls, plus FP4Q_ERR_ARG for a workspace that is too small
+ * and FP4Q_ERR_CUDA if the device cannot run a cooperative launch.  An empty
+ * tensor only zeroes *d_amax.  The paper has no counterpart of the workspace:
+ * it is how one launch replaces two.
+ */
+fp4q_status fp4q_nvfp4_sweep_dynamic(const void* x, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                     const float* importance, float* d_amax, uint8_t* codes,
+                                     uint8_t* scales_e4m3, float* d_global_scale, void* deq,
+                                     float* block_loss, void* workspace, size_t workspace_bytes,
+                                     int32_t* d_status, fp4q_stream_t stream);
+
+/*
  * fp4q_quantize_batch -- fp4q_quantize_dual for a list of weights, in one
  * persistent launch per FP4Q_BATCH_MAX weights.
  * Thread blocks take 16384-element tiles from a device queue ordered

@@ -110,6 +110,29 @@ def test_batch_argument_errors_without_a_gpu(fq):
     assert lib.fp4q_quantize_batch(arr, 0, 1, None, 0, None, None) == fq.OK
 
 
+def test_dynamic_argument_errors_without_a_gpu(fq):
+    lib = fq.load()
+    buf = ctypes.create_string_buffer(256)
+    p = ctypes.addressof(buf)
+    p16 = p + (-p % 16)
+    ws = fq.fp4q_dynamic_workspace_bytes()
+    assert ws >= 12
+
+    def call(x=p16, dt=1, rows=1, cols=16, imp=None, amax=p16, wsp=p16, nbytes=ws):
+        return lib.fp4q_nvfp4_sweep_dynamic(x, dt, rows, cols, imp, amax, p16, p16, p16, None, None,
+                                            wsp, nbytes, p16, None)
+
+    assert call(dt=7) == fq.ERR_DTYPE
+    assert call(cols=24) == fq.ERR_SHAPE
+    assert call(amax=None) == fq.ERR_NULL
+    assert call(x=None) == fq.ERR_NULL
+    assert call(wsp=None) == fq.ERR_NULL
+    assert call(x=p16 + 2) == fq.ERR_ALIGN
+    assert call(wsp=p16 + 4) == fq.ERR_ALIGN
+    assert call(imp=p16 + 4) == fq.ERR_ALIGN
+    assert call(nbytes=ws - 1) == fq.ERR_ARG
+
+
 def test_binding_refuses_cpu_tensors(fq):
     w = torch.zeros((4, 32), dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
