@@ -28,6 +28,7 @@ __all__ = [
     "fp4q_probe_e2m1", "fp4q_probe_e4m3",
     "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_quantize_batch_static", "BatchTensor",
     "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes", "nvfp4_quantize_dynamic",
+    "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout", "mma_scales",
     "quantize_batch",
     "NVFP4Result", "MXFP4Result", "nvfp4_quantize", "mxfp4_quantize", "quantize_dual", "dequantize",
     "FLAG_NONFINITE", "FLAG_RANGE", "FLAG_TIMEOUT",
@@ -47,7 +48,8 @@ EXPORTS = ("fp4q_version", "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_g
            "fp4q_nvfp4_sweepmse", "fp4q_nvfp4_sweepwmse", "fp4q_mxfp4_quant",
            "fp4q_mxfp4_quant_hadamard", "fp4q_mxfp4_quant_absmax", "fp4q_quantize_dual",
            "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_quantize_batch_static", "fp4q_dequant",
-           "fp4q_probe_e2m1", "fp4q_probe_e4m3", "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes")
+           "fp4q_probe_e2m1", "fp4q_probe_e4m3", "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes",
+           "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout")
 
 
 class BatchTensor(ctypes.Structure):
@@ -105,6 +107,7 @@ def load():
     }
     sigs["fp4q_quantize_batch"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, ctypes.c_size_t, P, P]
     sigs["fp4q_quantize_batch_static"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, P]
+    sigs["fp4q_scales_to_mma_layout"] = [P, I64, I64, P, P]
     sigs["fp4q_nvfp4_sweep_dynamic"] = [P, I, I64, I64, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -112,6 +115,8 @@ def load():
         fn.argtypes = args
     lib.fp4q_batch_workspace_bytes.restype = ctypes.c_size_t
     lib.fp4q_batch_workspace_bytes.argtypes = []
+    lib.fp4q_mma_scale_bytes.restype = I64
+    lib.fp4q_mma_scale_bytes.argtypes = [I64, I64]
     lib.fp4q_dynamic_workspace_bytes.restype = ctypes.c_size_t
     lib.fp4q_dynamic_workspace_bytes.argtypes = []
     _lib = lib
@@ -260,6 +265,29 @@ def fp4q_quantize_dual(w, importance, sign_masks, d_amax, nv_codes, nv_scales, d
     mp = _dev(sign_masks, "sign_masks", (torch.int32, torch.uint32), cols // MXFP4_BLOCK, w.device)
     _check(load().fp4q_quantize_dual(wp, _wdtype(w), rows, cols, ip, mp, ap, ncp, nsp, gp, ndp, nlp,
                                      cp, sp, dp, lp, st, _stream(stream)), "fp4q_quantize_dual")
+
+
+def fp4q_mma_scale_bytes(rows: int, scale_cols: int) -> int:
+    return int(load().fp4q_mma_scale_bytes(int(rows), int(scale_cols)))
+
+
+def fp4q_scales_to_mma_layout(scales: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """[rows][scale_cols] uint8 block scales -> the 128 x 4 tiled layout of
+    Blackwell block-scaled GEMMs, written to `out` (uint8, fp4q_mma_scale_bytes)."""
+    if scales.dim() != 2:
+        raise ValueError("scales must be a 2-D [rows][scale_cols] tensor")
+    rows, scols = scales.shape
+    sp = _dev(scales, "scales", torch.uint8, device=scales.device)
+    op = _dev(out, "out", torch.uint8, fp4q_mma_scale_bytes(rows, scols), scales.device)
+    _check(load().fp4q_scales_to_mma_layout(sp, rows, scols, op, _stream(stream)), "fp4q_scales_to_mma_layout")
+
+
+def mma_scales(scales: torch.Tensor, stream=None) -> torch.Tensor:
+    """Allocating form of fp4q_scales_to_mma_layout (flat uint8 tensor)."""
+    rows, scols = scales.shape
+    out = torch.empty(fp4q_mma_scale_bytes(rows, scols), dtype=torch.uint8, device=scales.device)
+    fp4q_scales_to_mma_layout(scales, out, stream)
+    return out
 
 
 def fp4q_dynamic_workspace_bytes() -> int:

@@ -236,6 +236,23 @@ fp4q_status fp4q_quantize_dual(const void* w, fp4q_dtype dt, int64_t rows, int64
                         d_global_scale, nv_deq, nv_loss, d_status, stream);
 }
 
+int64_t fp4q_mma_scale_bytes(int64_t rows, int64_t scale_cols)
+{
+    if (rows < 0 || scale_cols < 0 || (scale_cols != 0 && rows > INT64_MAX / 1024 / scale_cols)) return -1;
+    return fp4q::mma_scale_bytes(rows, scale_cols);
+}
+
+fp4q_status fp4q_scales_to_mma_layout(const uint8_t* scales, int64_t rows, int64_t scale_cols, uint8_t* out,
+                                      fp4q_stream_t stream)
+{
+    if (fp4q_mma_scale_bytes(rows, scale_cols) < 0) return FP4Q_ERR_SHAPE;
+    if (rows == 0 || scale_cols == 0) return FP4Q_OK;
+    if (!scales || !out) return FP4Q_ERR_NULL;
+    if (!aligned(out, 16)) return FP4Q_ERR_ALIGN;
+    fp4q::launch_mma_scale_layout(scales, rows, scale_cols, out, reinterpret_cast<cudaStream_t>(stream));
+    return after_launch();
+}
+
 size_t fp4q_dynamic_workspace_bytes(void) { return 16; }
 
 fp4q_status fp4q_nvfp4_sweep_dynamic(const void* x, fp4q_dtype dt, int64_t rows, int64_t cols,

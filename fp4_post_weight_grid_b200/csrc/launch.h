@@ -49,6 +49,10 @@ cudaError_t launch_nvfp4_dynamic(const void* w, bool bf16, int64_t rows, int64_t
                                  float* d_amax, uint8_t* codes, uint8_t* scales, float* d_S, void* deq,
                                  float* loss, unsigned* ws, int32_t* d_status, cudaStream_t s);
 
+// Block scales [rows][scols] -> the 128 x 4 tiled layout of block-scaled GEMMs.
+int64_t mma_scale_bytes(int64_t rows, int64_t scols);
+void launch_mma_scale_layout(const uint8_t* s, int64_t rows, int64_t scols, uint8_t* out, cudaStream_t st);
+
 void launch_dequant(bool mx, const uint8_t* codes, const uint8_t* scales, const float* d_S,
                     int64_t rows, int64_t cols, void* out, bool out_bf16, cudaStream_t s);
 

@@ -234,6 +234,36 @@ fp4q_status fp4q_quantize_dual(const void* w, fp4q_dtype dt, int64_t rows, int64
                                void* mx_deq, float* mx_loss, int32_t* d_status, fp4q_stream_t stream);
 
 /*
+ * fp4q_mma_scale_bytes -- bytes of the tiled scale layout written by
+ * fp4q_scales_to_mma_layout for a [rows][scale_cols] scale matrix:
+ * ceil(rows/128) * ceil(scale_cols/4) * 512; -1 for a negative or
+ * overflowing size.
+ */
+int64_t fp4q_mma_scale_bytes(int64_t rows, int64_t scale_cols);
+
+/*
+ * fp4q_scales_to_mma_layout -- block scales in the layout that Blackwell
+ * block-scaled FP4 GEMMs read (the MR-GPTQ summary, technical sec. 3, runs the
+ * quantized weights through such kernels; the pages do not describe the
+ * layout, it is the hardware's).  The [rows][scale_cols] matrix of scale
+ * bytes (E4M3 for NVFP4 with scale_cols = cols/16, E8M0 for MXFP4 with
+ * scale_cols = cols/32, as written by the quantizers above) is cut into tiles
+ * of 128 rows x 4 scale columns, zero-padded at the bottom and right edges;
+ * tiles are stored one after the other, the column tiles of one row tile
+ * together; inside a 512-byte tile the byte of (row r, column c) is at
+ * (r % 32) * 16 + (r / 32) * 4 + c.  The packed codes need no change: their
+ * row-major nibble order (element 2j in the low nibble of byte j) is the
+ * K-major operand order of those GEMMs.
+ *   scales  device, rows * scale_cols bytes, row-major.
+ *   out     device, 16-byte aligned, fp4q_mma_scale_bytes(rows, scale_cols)
+ *           bytes, fully written (padding zeroed).
+ * Errors: FP4Q_ERR_SHAPE (negative sizes), FP4Q_ERR_NULL, FP4Q_ERR_ALIGN; an
+ * empty matrix touches nothing.
+ */
+fp4q_status fp4q_scales_to_mma_layout(const uint8_t* scales, int64_t rows, int64_t scale_cols, uint8_t* out,
+                                      fp4q_stream_t stream);
+
+/*
  * fp4q_dynamic_workspace_bytes -- size of the workspace of
  * fp4q_nvfp4_sweep_dynamic (16 bytes).
  */

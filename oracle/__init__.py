@@ -17,7 +17,11 @@ stated in ``fp4q_oracle.c``.
 Parity pins: the functions here are pinned by tests/test_oracle_codecs.py,
 tests/test_oracle_nvfp4.py and tests/test_oracle_mxfp4.py.  The optimality of
 the MXFP4 exponent window e0-1..e0+1 is not claimed by the pages and is
-"parity unpinned" beyond the defined computation.
+"parity unpinned" beyond the defined computation.  ``scales_to_mma_layout``
+(the tiled scale layout read by Blackwell block-scaled GEMMs, a hardware
+interface the pages do not describe) is "parity unpinned" on the CPU: only its
+size and zero padding are checked there, and a library GEMM that reads the
+layout pins it on the GPU (tests/test_gpu_mma_layout.py).
 """
 from __future__ import annotations
 
@@ -83,6 +87,8 @@ def _load():
             "orc_mxfp4_quant": (I, [P, I64, I64, P, P, P, P, P, P, I]),
             "orc_mxfp4_dequant": (None, [P, P, I64, I64, P]),
             "orc_max_threads": (I, []),
+            "orc_mma_scale_bytes": (I64, [I64, I64]),
+            "orc_scales_to_mma_layout": (None, [P, I64, I64, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -262,6 +268,15 @@ def mxfp4_dequant(codes: np.ndarray, scales: np.ndarray, rows: int, cols: int) -
     y = np.empty((rows, cols), dtype=np.float32)
     _load().orc_mxfp4_dequant(_ptr(codes), _ptr(scales), rows, cols, _ptr(y))
     return y
+
+
+def scales_to_mma_layout(scales: np.ndarray) -> np.ndarray:
+    """[rows][scols] block-scale bytes -> the 128 x 4 tiled layout (flat uint8)."""
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, scols = scales.shape
+    out = np.empty(int(_load().orc_mma_scale_bytes(rows, scols)), dtype=np.uint8)
+    _load().orc_scales_to_mma_layout(_ptr(scales), rows, scols, _ptr(out))
+    return out
 
 
 def max_threads() -> int:

@@ -37,6 +37,8 @@
  * codec sweeps against nearest-value search, the 126-value count, the window
  * ratios of Lemmas 4.1/4.3, brute force over all 126 scales, closed forms,
  * fp64 recomputation of losses, the dense Sylvester Hadamard matrix).
+ * orc_scales_to_mma_layout is parity unpinned on the CPU (a hardware layout
+ * the pages do not describe); a library GEMM reading it pins it on the GPU.
  */
 #include <math.h>
 #include <stdint.h>
@@ -471,6 +473,41 @@ void orc_mxfp4_dequant(const uint8_t* codes, const uint8_t* scales,
     for (i = 0; i < n; ++i) {
         int nib = (codes[i / 2] >> ((i % 2) * 4)) & 15;
         y[i] = orc_e2m1_decode(nib) * orc_e8m0_value(scales[i / 32]);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Block scales in the layout of Blackwell block-scaled FP4 GEMMs            */
+/* ------------------------------------------------------------------------ */
+
+/* [MR] sec. 3 runs the quantized weights through block-scaled FP4 GEMM
+ * kernels on Blackwell.  Those read the block scales of an operand not row by
+ * row but in tiles: the [rows][scols] scale matrix (scols = cols/16 for
+ * NVFP4, cols/32 for MXFP4) is cut into tiles of 128 rows x 4 scale columns,
+ * zero-padded at the bottom and right edges, and the tiles are stored one
+ * after the other, the column tiles of one row tile together.  A tile is 512
+ * bytes: 32 lines of 16 bytes, line j holding rows j, j+32, j+64, j+96 of the
+ * tile, 4 scale bytes each.  This is a hardware interface, not part of the
+ * method; the pages do not describe it.  Parity pinned on the GPU only: a
+ * library block-scaled GEMM reads this layout in tests/test_gpu_mma_layout.py;
+ * on the CPU only its shape and its zero padding are checked. */
+int64_t orc_mma_scale_bytes(int64_t rows, int64_t scols)
+{
+    return ((rows + 127) / 128) * ((scols + 3) / 4) * 512;
+}
+
+void orc_scales_to_mma_layout(const uint8_t* s, int64_t rows, int64_t scols, uint8_t* out)
+{
+    int64_t r, c;
+    int64_t col_tiles = (scols + 3) / 4;
+    memset(out, 0, (size_t)orc_mma_scale_bytes(rows, scols));
+    for (r = 0; r < rows; ++r) {
+        for (c = 0; c < scols; ++c) {
+            int64_t tile = (r / 128) * col_tiles + c / 4;
+            int64_t line = r % 32;
+            int64_t slot = (r % 128) / 32;
+            out[tile * 512 + line * 16 + slot * 4 + c % 4] = s[r * scols + c];
+        }
     }
 }
 

@@ -155,3 +155,19 @@ def test_mxfp4_dequant_reproduces_reconstruction(orc):
     out = orc.mxfp4_quant(x, sign_masks=synth.sign_masks(256, seed=1))
     y = orc.mxfp4_dequant(out["codes"], out["scales"], 16, 256)
     np.testing.assert_array_equal(y, out["y"])
+
+
+# ---------------------------------------------------------------- tiled scale layout
+# The layout itself is a hardware interface the pages do not describe ("parity
+# unpinned" on the CPU): a library GEMM pins it on the GPU.  Here: its size, that
+# every input byte lands exactly once, and that the padding is zero.
+
+@pytest.mark.parametrize("rows,scols", [(1, 1), (128, 4), (130, 6), (300, 257), (4096, 256)])
+def test_mma_layout_size_coverage_and_padding(orc, rows, scols):
+    rng = np.random.default_rng(rows * 1000 + scols)
+    s = rng.integers(1, 256, size=(rows, scols), dtype=np.uint8)     # no zero bytes in the input
+    out = orc.scales_to_mma_layout(s)
+    rt, ct = -(-rows // 128), -(-scols // 4)
+    assert out.size == rt * ct * 512
+    assert np.count_nonzero(out) == rows * scols                      # padding is zero
+    assert sorted(out[out != 0].tolist()) == sorted(s.reshape(-1).tolist())
