@@ -382,6 +382,7 @@ SINGLE_PATHS = {
     "mxfp4-absmax": (B_MXFP4, "mxfp4_kernel with the fused global max"),
     "mxfp4-hadamard": (B_MXFP4, "mxfp4_kernel Hadamard"),
     "dequant-nvfp4": (0.5 + 1.0 / 16 + 2.0, "dequant_kernel NVFP4"),
+    "mma-layout": (2.0 / 16, "mma_scale_layout_kernel (NVFP4 scales, read + write)"),
 }
 
 
@@ -407,6 +408,7 @@ def run_single(args):
     sc16 = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
     sc32 = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
     deq = torch.empty_like(w)
+    tiled = torch.empty(fq.fp4q_mma_scale_bytes(rows, cols // 16), dtype=torch.uint8, device=dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     fq.fp4q_global_absmax(w, amax)
     fq.fp4q_nvfp4_sweepmse(w, amax, codes, sc16, S, deq, None, st)
@@ -425,6 +427,8 @@ def run_single(args):
             fq.fp4q_mxfp4_quant_absmax(w, None, codes, sc32, amax, deq, None, st, stream)
         elif args.single == "mxfp4-hadamard":
             fq.fp4q_mxfp4_quant_hadamard(w, masks, codes, sc32, deq, None, st, stream)
+        elif args.single == "mma-layout":
+            fq.fp4q_scales_to_mma_layout(sc16, tiled, stream)
         elif args.single == "dequant-nvfp4":
             fq.fp4q_dequant(fq.NVFP4, codes, sc16, S, rows, cols, deq, stream)
 
