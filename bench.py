@@ -311,6 +311,22 @@ def cpu_baseline(seconds_hint=20.0):
             "elements_per_s": n / dt}
 
 
+def rank_seed(rank: int) -> int:
+    """Seed of the replica on `rank`: every rank quantizes its own synthetic
+    copy of the workload (weak scaling), drawn from seed 5 + 1000 * rank."""
+    return 5 + 1000 * rank
+
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's time: an all-reduce (MAX) over the process group, or
+    `ms` itself without one."""
+    if dist is None:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_reference(args):
     """--impl reference: the CPU oracle timed on the host cores, per step one bounded
     sample of the workload (see cpu_baseline)."""
@@ -569,11 +585,11 @@ def main():
         import torch.distributed as dist
         from datetime import timedelta
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
 
-    model = Model(fq, dev, seed=5 + 1000 * rank, with_events=True)
+    model = Model(fq, dev, seed=rank_seed(rank), with_events=True)
     stream = torch.cuda.Stream(device=dev)
     streams = [stream] + [torch.cuda.Stream(device=dev) for _ in range(args.streams - 1)]
     stream.wait_stream(torch.cuda.current_stream())
@@ -619,10 +635,7 @@ def main():
         dist.barrier()
     clk = clocks.stop()
     ms = t_start.elapsed_time(t_end) / args.steps
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, dev)
     status = int(model.status.item())
 
     hbm_peak, peak_kind, sm_max = load_peaks()
