@@ -88,6 +88,9 @@ def _load():
             "orc_mxfp4_dequant": (None, [P, P, I64, I64, P]),
             "orc_max_threads": (I, []),
             "orc_mma_scale_bytes": (I64, [I64, I64]),
+            "orc_hadamard32_inverse": (None, [P, ctypes.c_uint32, P]),
+            "orc_mxfp4_unrotate": (None, [P, I64, I64, P, P]),
+            "orc_focus_quant": (I, [I, P, I64, I64, P, F, P, I, P, P, P]),
             "orc_scales_to_mma_layout": (None, [P, I64, I64, P]),
         }
         for name, (res, args) in sigs.items():
@@ -268,6 +271,42 @@ def mxfp4_dequant(codes: np.ndarray, scales: np.ndarray, rows: int, cols: int) -
     y = np.empty((rows, cols), dtype=np.float32)
     _load().orc_mxfp4_dequant(_ptr(codes), _ptr(scales), rows, cols, _ptr(y))
     return y
+
+
+def hadamard32_inverse(y: np.ndarray, mask: int) -> np.ndarray:
+    y = _f32(y).reshape(32)
+    x = np.empty(32, dtype=np.float32)
+    _load().orc_hadamard32_inverse(_ptr(y), ctypes.c_uint32(int(mask) & 0xFFFFFFFF), _ptr(x))
+    return x
+
+
+def mxfp4_unrotate(y: np.ndarray, sign_masks: np.ndarray) -> np.ndarray:
+    """Rotated-domain rows x cols values back to the original domain."""
+    y = _f32(y)
+    rows, cols = y.shape
+    m = np.ascontiguousarray(sign_masks, dtype=np.uint32)
+    x = np.empty((rows, cols), dtype=np.float32)
+    _load().orc_mxfp4_unrotate(_ptr(y), rows, cols, _ptr(m), _ptr(x))
+    return x
+
+
+def focus_quant(fmt: int, x: np.ndarray, scales: np.ndarray, coeffs: np.ndarray, sub: int, S=1.0) -> dict:
+    """FOCUS forward quantizer: codes of x / (S_dq * c_k) with the given block
+    scales (fmt 0 NVFP4 E4M3 patterns + global S, 1 MXFP4 E8M0 bytes) and the
+    per-sub-block coefficients `coeffs` (fp16 or fp32 values, one per `sub`
+    elements); the reconstruction uses S_dq."""
+    x = _f32(x)
+    rows, cols = x.shape
+    bs = NVFP4_BLOCK if fmt == 0 else MXFP4_BLOCK
+    scales = np.ascontiguousarray(scales, dtype=np.uint8).reshape(-1)
+    c = np.ascontiguousarray(np.asarray(coeffs).astype(np.float32)).reshape(-1)   # fp16 -> fp32 is exact
+    assert scales.size == rows * cols // bs and c.size == rows * cols // sub
+    codes = np.empty(rows * cols // 2, dtype=np.uint8)
+    y = np.empty((rows, cols), dtype=np.float32)
+    loss = np.empty(rows * cols // bs, dtype=np.float32)
+    st = _load().orc_focus_quant(int(fmt), _ptr(x), rows, cols, _ptr(scales), float(np.float32(S)), _ptr(c),
+                                 int(sub), _ptr(codes), _ptr(y), _ptr(loss))
+    return {"status": st, "codes": codes.reshape(rows, cols // 2), "y": y, "loss": loss.reshape(rows, cols // bs)}
 
 
 def scales_to_mma_layout(scales: np.ndarray) -> np.ndarray:

@@ -476,6 +476,109 @@ void orc_mxfp4_dequant(const uint8_t* codes, const uint8_t* scales,
     }
 }
 
+/* Inverse of orc_hadamard32: x = sigma o (c * H32 * y).  (c*H32)^2 = I in
+ * exact arithmetic (H32 symmetric, H32^2 = 32 I, c = 1/sqrt(32)) and
+ * sigma o sigma = 1, so the same five butterfly stages h = 1,2,4,8,16, then
+ * the multiply by c, then the sign flips, undo the rotation up to rounding
+ * ([MR] sec. 2: the deployed weights live in the rotated domain; this maps a
+ * reconstruction back to the original one). */
+void orc_hadamard32_inverse(const float* y, uint32_t mask, float* x)
+{
+    int i, h;
+    float c = orc_hadamard_scale();
+    float v[32];
+    for (i = 0; i < 32; ++i) v[i] = y[i];
+    for (h = 1; h < 32; h *= 2) {
+        for (i = 0; i < 32; ++i) {
+            if (i & h) continue;
+            {
+                float a = v[i], b = v[i + h];
+                v[i] = a + b;
+                v[i + h] = a - b;
+            }
+        }
+    }
+    for (i = 0; i < 32; ++i) {
+        float t = v[i] * c;
+        x[i] = ((mask >> i) & 1u) ? -t : t;
+    }
+}
+
+/* Rows x cols (cols % 32 == 0) of rotated-domain values back to the original
+ * domain, block by block (sign_masks[cols/32] as in orc_mxfp4_quant). */
+void orc_mxfp4_unrotate(const float* y, int64_t rows, int64_t cols, const uint32_t* sign_masks, float* x)
+{
+    int64_t r, b, nb = cols / 32;
+    for (r = 0; r < rows; ++r)
+        for (b = 0; b < nb; ++b)
+            orc_hadamard32_inverse(y + r * cols + b * 32, sign_masks[b], x + r * cols + b * 32);
+}
+
+/* ------------------------------------------------------------------------ */
+/* FOCUS forward quantizer  ([FC] "Metodologia" 2-3)                          */
+/* ------------------------------------------------------------------------ */
+
+/* Quantize with a quantization scale decoupled from the stored one.  [FC]
+ * keeps the hardware dequantization scale S_dq of every block (E4M3 x S for
+ * NVFP4, E8M0 for MXFP4) and quantizes sub-block k of the block with
+ * S_q = S_dq * c_k, c_k a full-precision coefficient (CRS: one per block;
+ * DGS: one per sub-block, e.g. 8 elements); the codes are Q(W_k / S_q) and
+ * the stored reconstruction is q * S_dq.  Reading taken (the page gives the
+ * formula only): with d = S_dq computed as everywhere else (NVFP4
+ * d = RN(E4M3(p) * S), MXFP4 d = 2^(b-127)),
+ *   dq_k = RN(d * c_k);  inv_k = RN(1 / dq_k)
+ *   r = x_i * inv_k;  q = E2M1(r);  y = RN(q * d);  e = x_i - y;  L = L + e*e
+ * with L the block's loss in column order.  fmt 0 = NVFP4 (16-element blocks,
+ * scales E4M3 patterns, S the global scale), 1 = MXFP4 (32, E8M0 bytes).
+ * coeffs[rows * cols / sub] (sub divides the block).  Returns ORC_RANGE if a
+ * scale byte is not a positive finite value (NVFP4 0x01..0x7E, MXFP4 not
+ * 0xFF) or a coefficient is not positive and finite, ORC_NONFINITE if an
+ * input is not finite; the outputs of such blocks are then unspecified. */
+int orc_focus_quant(int fmt, const float* x, int64_t rows, int64_t cols, const uint8_t* scales, float S,
+                    const float* coeffs, int sub, uint8_t* codes, float* y, float* loss)
+{
+    const int bs = fmt == 0 ? 16 : 32;
+    int64_t nb = cols / bs, r;
+    int status = ORC_OK;
+    if (cols % bs || sub <= 0 || bs % sub) return 2;
+    for (r = 0; r < rows; ++r) {
+        int64_t b;
+        for (b = 0; b < nb; ++b) {
+            const float* xb = x + r * cols + b * bs;
+            int64_t blk = r * nb + b;
+            int i, sb = scales[blk];
+            uint8_t nib[32];
+            float d, L = 0.0f;
+            if (fmt == 0) {
+                if (sb < 1 || sb > 126) status = ORC_RANGE;
+                d = orc_e4m3_value(sb) * S;
+            } else {
+                if (sb == 255) status = ORC_RANGE;
+                d = orc_e8m0_value(sb);
+            }
+            for (i = 0; i < bs; ++i) {
+                float c = coeffs[(r * cols + b * bs + i) / sub];
+                float dq = d * c;
+                float inv = 1.0f / dq;
+                float rr = xb[i] * inv;
+                int code = orc_e2m1_encode(rr);
+                float q = orc_e2m1_decode(code);
+                float yy = q * d;
+                float e = xb[i] - yy;
+                float e2 = e * e;
+                if (!(c > 0.0f) || isinf(c)) status = ORC_RANGE;
+                if (!isfinite(xb[i]) && status == ORC_OK) status = ORC_NONFINITE;
+                L = L + e2;
+                nib[i] = (uint8_t)code;
+                if (y) y[r * cols + b * bs + i] = yy;
+            }
+            if (codes) pack_nibbles(nib, bs, codes + blk * (bs / 2));
+            if (loss) loss[blk] = L;
+        }
+    }
+    return status;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Block scales in the layout of Blackwell block-scaled FP4 GEMMs            */
 /* ------------------------------------------------------------------------ */
