@@ -399,6 +399,9 @@ SINGLE_PATHS = {
     "mxfp4-hadamard": (B_MXFP4, "mxfp4_kernel Hadamard"),
     "dequant-nvfp4": (0.5 + 1.0 / 16 + 2.0, "dequant_kernel NVFP4"),
     "mma-layout": (2.0 / 16, "mma_scale_layout_kernel (NVFP4 scales, read + write)"),
+    "focus-nvfp4": (2.0 + 1.0 / 16 + 2.0 / 8 + 0.5 + 2.0, "focus_kernel NVFP4, sub-blocks of 8"),
+    "focus-mxfp4": (2.0 + 1.0 / 32 + 2.0 / 8 + 0.5 + 2.0, "focus_kernel MXFP4, sub-blocks of 8"),
+    "unrotate": (4.0, "unrotate_kernel (MXFP4 Hadamard inverse, bf16 in and out)"),
 }
 
 
@@ -425,9 +428,11 @@ def run_single(args):
     sc32 = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
     deq = torch.empty_like(w)
     tiled = torch.empty(fq.fp4q_mma_scale_bytes(rows, cols // 16), dtype=torch.uint8, device=dev)
+    coeffs = (1.0 + 0.25 * torch.rand((rows, cols // 8), device=dev)).to(torch.float16)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     fq.fp4q_global_absmax(w, amax)
     fq.fp4q_nvfp4_sweepmse(w, amax, codes, sc16, S, deq, None, st)
+    fq.fp4q_mxfp4_quant(w, codes, sc32, None, None, st)
     stream = torch.cuda.current_stream()
 
     def launch():
@@ -443,6 +448,12 @@ def run_single(args):
             fq.fp4q_mxfp4_quant_absmax(w, None, codes, sc32, amax, deq, None, st, stream)
         elif args.single == "mxfp4-hadamard":
             fq.fp4q_mxfp4_quant_hadamard(w, masks, codes, sc32, deq, None, st, stream)
+        elif args.single == "focus-nvfp4":
+            fq.fp4q_focus_quant(fq.NVFP4, w, sc16, S, coeffs, 8, codes, deq, None, st, stream)
+        elif args.single == "focus-mxfp4":
+            fq.fp4q_focus_quant(fq.MXFP4, w, sc32, None, coeffs, 8, codes, deq, None, st, stream)
+        elif args.single == "unrotate":
+            fq.fp4q_mxfp4_unrotate(w, masks, deq, stream)
         elif args.single == "mma-layout":
             fq.fp4q_scales_to_mma_layout(sc16, tiled, stream)
         elif args.single == "dequant-nvfp4":

@@ -29,6 +29,7 @@ __all__ = [
     "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_quantize_batch_static", "BatchTensor",
     "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes", "nvfp4_quantize_dynamic",
     "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout", "mma_scales",
+    "fp4q_focus_quant", "fp4q_mxfp4_unrotate", "focus_quantize", "mxfp4_unrotate", "FocusResult",
     "quantize_batch",
     "NVFP4Result", "MXFP4Result", "nvfp4_quantize", "mxfp4_quantize", "quantize_dual", "dequantize",
     "FLAG_NONFINITE", "FLAG_RANGE", "FLAG_TIMEOUT",
@@ -49,7 +50,7 @@ EXPORTS = ("fp4q_version", "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_g
            "fp4q_mxfp4_quant_hadamard", "fp4q_mxfp4_quant_absmax", "fp4q_quantize_dual",
            "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_quantize_batch_static", "fp4q_dequant",
            "fp4q_probe_e2m1", "fp4q_probe_e4m3", "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes",
-           "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout")
+           "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout", "fp4q_focus_quant", "fp4q_mxfp4_unrotate")
 
 
 class BatchTensor(ctypes.Structure):
@@ -108,6 +109,8 @@ def load():
     sigs["fp4q_quantize_batch"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, ctypes.c_size_t, P, P]
     sigs["fp4q_quantize_batch_static"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, P]
     sigs["fp4q_scales_to_mma_layout"] = [P, I64, I64, P, P]
+    sigs["fp4q_focus_quant"] = [I, P, I, I64, I64, P, P, P, ctypes.c_int32, P, P, P, P, P]
+    sigs["fp4q_mxfp4_unrotate"] = [P, I, I64, I64, P, P, P]
     sigs["fp4q_nvfp4_sweep_dynamic"] = [P, I, I64, I64, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -265,6 +268,38 @@ def fp4q_quantize_dual(w, importance, sign_masks, d_amax, nv_codes, nv_scales, d
     mp = _dev(sign_masks, "sign_masks", (torch.int32, torch.uint32), cols // MXFP4_BLOCK, w.device)
     _check(load().fp4q_quantize_dual(wp, _wdtype(w), rows, cols, ip, mp, ap, ncp, nsp, gp, ndp, nlp,
                                      cp, sp, dp, lp, st, _stream(stream)), "fp4q_quantize_dual")
+
+
+def fp4q_focus_quant(fmt: int, w, scales, d_global_scale, coeffs, sub_block: int, codes, deq=None,
+                     block_loss=None, d_status=None, stream=None) -> None:
+    """FOCUS forward quantizer: codes of w / (S_dq * c_k) per sub-block, the
+    reconstruction with S_dq.  `scales`: the stored block scale bytes;
+    `coeffs`: float16 [rows, cols / sub_block]; `d_global_scale`: NVFP4 S."""
+    bs = MXFP4_BLOCK if fmt == MXFP4 else NVFP4_BLOCK
+    rows, cols = _rc(w, bs)
+    dev = w.device
+    n = rows * cols
+    sub = int(sub_block)
+    if sub <= 0 or bs % sub:
+        raise Fp4qError(ERR_ARG, f"fp4q_focus_quant: sub_block {sub} does not divide the block of {bs}")
+    args = (_dev(w, "w", device=dev), _wdtype(w), rows, cols,
+            _dev(scales, "scales", torch.uint8, n // bs, dev),
+            _dev(d_global_scale, "d_global_scale", torch.float32, 1, dev),
+            _dev(coeffs, "coeffs", torch.float16, n // sub, dev), sub,
+            _dev(codes, "codes", torch.uint8, n // 2, dev), _dev(deq, "deq", w.dtype, n, dev),
+            _dev(block_loss, "block_loss", torch.float32, n // bs, dev),
+            _dev(d_status, "d_status", torch.int32, 1, dev), _stream(stream))
+    _check(load().fp4q_focus_quant(int(fmt), *args), "fp4q_focus_quant")
+
+
+def fp4q_mxfp4_unrotate(y, sign_masks, out, stream=None) -> None:
+    """Rotated-domain MXFP4 reconstruction `y` back to the original domain, into `out`."""
+    rows, cols = _rc(y, MXFP4_BLOCK)
+    dev = y.device
+    _check(load().fp4q_mxfp4_unrotate(_dev(y, "y", device=dev), _wdtype(y), rows, cols,
+                                      _dev(sign_masks, "sign_masks", (torch.int32, torch.uint32), cols // 32, dev),
+                                      _dev(out, "out", y.dtype, rows * cols, dev), _stream(stream)),
+           "fp4q_mxfp4_unrotate")
 
 
 def fp4q_mma_scale_bytes(rows: int, scale_cols: int) -> int:
@@ -480,6 +515,35 @@ def nvfp4_quantize_dynamic(x: torch.Tensor, importance: Optional[torch.Tensor] =
         workspace = torch.zeros(fp4q_dynamic_workspace_bytes() // 4, dtype=torch.int32, **kw)
     fp4q_nvfp4_sweep_dynamic(x, importance, amax, codes, scales, S, deq, loss, workspace, status, stream)
     return NVFP4Result(codes, scales, S, deq, loss, amax, status)
+
+
+class FocusResult(NamedTuple):
+    codes: torch.Tensor           # uint8 [rows, cols/2]
+    deq: Optional[torch.Tensor]   # reconstruction with the stored scales
+    block_loss: Optional[torch.Tensor]
+    status: torch.Tensor
+
+
+def focus_quantize(w: torch.Tensor, fmt: int, scales: torch.Tensor, coeffs: torch.Tensor, sub_block: int = 8,
+                   global_scale: Optional[torch.Tensor] = None, with_deq=True, with_loss=True,
+                   stream=None) -> FocusResult:
+    """Allocating form of fp4q_focus_quant."""
+    bs = MXFP4_BLOCK if fmt == MXFP4 else NVFP4_BLOCK
+    rows, cols = _rc(w, bs)
+    kw = dict(device=w.device)
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, **kw)
+    deq = torch.empty_like(w) if with_deq else None
+    loss = torch.empty((rows, cols // bs), dtype=torch.float32, **kw) if with_loss else None
+    status = torch.zeros(1, dtype=torch.int32, **kw)
+    fp4q_focus_quant(fmt, w, scales, global_scale, coeffs, sub_block, codes, deq, loss, status, stream)
+    return FocusResult(codes, deq, loss, status)
+
+
+def mxfp4_unrotate(y: torch.Tensor, sign_masks: torch.Tensor, stream=None) -> torch.Tensor:
+    """Allocating form of fp4q_mxfp4_unrotate."""
+    out = torch.empty_like(y)
+    fp4q_mxfp4_unrotate(y, sign_masks, out, stream)
+    return out
 
 
 def mxfp4_quantize(w: torch.Tensor, sign_masks: Optional[torch.Tensor] = None, with_deq=True,

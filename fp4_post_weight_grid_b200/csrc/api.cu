@@ -236,6 +236,39 @@ fp4q_status fp4q_quantize_dual(const void* w, fp4q_dtype dt, int64_t rows, int64
                         d_global_scale, nv_deq, nv_loss, d_status, stream);
 }
 
+fp4q_status fp4q_focus_quant(fp4q_format fmt, const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                             const uint8_t* scales, const float* d_global_scale, const void* coeffs_f16,
+                             int32_t sub_block, uint8_t* codes, void* deq, float* block_loss, int32_t* d_status,
+                             fp4q_stream_t stream)
+{
+    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_DTYPE;
+    const bool mx = fmt == FP4Q_MXFP4;
+    const int64_t bs = mx ? FP4Q_MXFP4_BLOCK : FP4Q_NVFP4_BLOCK;
+    if (!(sub_block == 4 || sub_block == 8 || sub_block == 16 || (mx && sub_block == 32))) return FP4Q_ERR_ARG;
+    bool empty = false;
+    fp4q_status st = check_quant_args(w, dt, rows, cols, bs, codes, scales, d_status, deq, block_loss,
+                                      mx ? 16 : 8, &empty);
+    if (st != FP4Q_OK || empty) return st;
+    if (!coeffs_f16 || (!mx && !d_global_scale)) return FP4Q_ERR_NULL;
+    if (!aligned(coeffs_f16, 2) || (!mx && !aligned(d_global_scale, 4))) return FP4Q_ERR_ALIGN;
+    if (!fp4q::launch_focus(mx, dt == FP4Q_BF16, sub_block, w, rows, cols, scales, d_global_scale, coeffs_f16,
+                            codes, deq, block_loss, d_status, reinterpret_cast<cudaStream_t>(stream)))
+        return FP4Q_ERR_ARG;
+    return after_launch();
+}
+
+fp4q_status fp4q_mxfp4_unrotate(const void* y, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                const uint32_t* sign_masks, void* out, fp4q_stream_t stream)
+{
+    if (!valid_dtype(dt)) return FP4Q_ERR_DTYPE;
+    if (!shape_ok(rows, cols, FP4Q_MXFP4_BLOCK)) return FP4Q_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return FP4Q_OK;
+    if (!y || !sign_masks || !out) return FP4Q_ERR_NULL;
+    if (!aligned(y, 16) || !aligned(out, 16) || !aligned(sign_masks, 4)) return FP4Q_ERR_ALIGN;
+    fp4q::launch_unrotate(dt == FP4Q_BF16, y, rows, cols, sign_masks, out, reinterpret_cast<cudaStream_t>(stream));
+    return after_launch();
+}
+
 int64_t fp4q_mma_scale_bytes(int64_t rows, int64_t scale_cols)
 {
     if (rows < 0 || scale_cols < 0 || (scale_cols != 0 && rows > INT64_MAX / 1024 / scale_cols)) return -1;

@@ -49,6 +49,16 @@ cudaError_t launch_nvfp4_dynamic(const void* w, bool bf16, int64_t rows, int64_t
                                  float* d_amax, uint8_t* codes, uint8_t* scales, float* d_S, void* deq,
                                  float* loss, unsigned* ws, int32_t* d_status, cudaStream_t s);
 
+// FOCUS forward quantizer (mx: MXFP4 blocks of 32, else NVFP4 blocks of 16),
+// sub in {4, 8, 16} (and 32 for MXFP4); false for an unsupported sub-block size.
+bool launch_focus(bool mx, bool bf16, int sub, const void* w, int64_t rows, int64_t cols, const uint8_t* scales,
+                  const float* d_S, const void* coeffs, uint8_t* codes, void* deq, float* loss,
+                  int32_t* d_status, cudaStream_t s);
+
+// Rotated-domain MXFP4 reconstruction back to the original domain.
+void launch_unrotate(bool bf16, const void* y, int64_t rows, int64_t cols, const uint32_t* sign_masks, void* out,
+                     cudaStream_t s);
+
 // Block scales [rows][scols] -> the 128 x 4 tiled layout of block-scaled GEMMs.
 int64_t mma_scale_bytes(int64_t rows, int64_t scols);
 void launch_mma_scale_layout(const uint8_t* s, int64_t rows, int64_t scols, uint8_t* out, cudaStream_t st);

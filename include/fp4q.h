@@ -234,6 +234,51 @@ fp4q_status fp4q_quantize_dual(const void* w, fp4q_dtype dt, int64_t rows, int64
                                void* mx_deq, float* mx_loss, int32_t* d_status, fp4q_stream_t stream);
 
 /*
+ * fp4q_focus_quant -- the FOCUS forward quantizer ("FOCUS" summary,
+ * gist.science, arXiv 2608.01847, "Metodologia" 2-3): quantize with a
+ * quantization scale decoupled from the stored one.  Each hardware block
+ * keeps its dequantization scale S_dq (NVFP4: E4M3 pattern p times the global
+ * scale S; MXFP4: E8M0 byte b, 2^(b-127)); sub-block k of sub_block elements
+ * is quantized with S_q = S_dq * c_k (CRS: sub_block = the block size; DGS: a
+ * smaller sub-block, e.g. 8), and the stored reconstruction uses S_dq:
+ *   d = RN(E4M3(p) * S) or 2^(b-127);  dq = RN(d * c_k);  inv = RN(1 / dq)
+ *   code = E2M1(RN(x * inv));  deq = RN(q * d);
+ *   block_loss = sum over the block, in column order, of RN(x - deq)^2.
+ * The codes with the given scales are a standard NVFP4/MXFP4 tensor (the
+ * coefficients are not stored).
+ *   fmt         FP4Q_NVFP4 (16-element blocks) or FP4Q_MXFP4 (32).
+ *   w, dt, rows, cols   as the quantizers (cols a multiple of the block).
+ *   scales      device, one byte per block (E4M3 patterns 0x01..0x7E or E8M0
+ *               bytes 0..254), row-major [rows][cols/block].
+ *   d_global_scale  device float S (NVFP4; ignored and may be NULL for MXFP4).
+ *   coeffs_f16  device, IEEE binary16 coefficients c_k, [rows][cols/sub_block],
+ *               2-byte aligned; must be positive and finite.
+ *   sub_block   4, 8 or 16 (and 32 for MXFP4).
+ *   codes, deq, block_loss  as the quantizers (deq, block_loss may be NULL).
+ * Errors: as the quantizers, FP4Q_ERR_ARG for another sub_block; on the
+ * device FP4Q_FLAG_RANGE for a scale byte or coefficient outside the allowed
+ * values and FP4Q_FLAG_NONFINITE for a NaN/Inf input (outputs of such blocks
+ * unspecified).
+ */
+fp4q_status fp4q_focus_quant(fp4q_format fmt, const void* w, fp4q_dtype dt, int64_t rows, int64_t cols,
+                             const uint8_t* scales, const float* d_global_scale, const void* coeffs_f16,
+                             int32_t sub_block, uint8_t* codes, void* deq, float* block_loss, int32_t* d_status,
+                             fp4q_stream_t stream);
+
+/*
+ * fp4q_mxfp4_unrotate -- map a rotated-domain MXFP4 reconstruction (the deq of
+ * fp4q_mxfp4_quant_hadamard) back to the original domain (MR-GPTQ summary,
+ * technical sec. 2).  Per 32-block: the five butterfly stages h = 1..16 of
+ * the rotation, every element times c = RN(1/sqrt(32)), then the sign flips
+ * of sign_masks; (c * H32)^2 = I, so this inverts the rotation up to rounding.
+ *   y, out      device, rows x cols of dt, 16-byte aligned (may not overlap).
+ *   sign_masks  device, cols/32 uint32 as for the rotation.
+ * cols % 32 == 0.  Errors as fp4q_mxfp4_quant_hadamard.
+ */
+fp4q_status fp4q_mxfp4_unrotate(const void* y, fp4q_dtype dt, int64_t rows, int64_t cols,
+                                const uint32_t* sign_masks, void* out, fp4q_stream_t stream);
+
+/*
  * fp4q_mma_scale_bytes -- bytes of the tiled scale layout written by
  * fp4q_scales_to_mma_layout for a [rows][scale_cols] scale matrix:
  * ceil(rows/128) * ceil(scale_cols/4) * 512; -1 for a negative or
