@@ -91,6 +91,7 @@ def _load():
             "orc_hadamard32_inverse": (None, [P, ctypes.c_uint32, P]),
             "orc_mxfp4_unrotate": (None, [P, I64, I64, P, P]),
             "orc_focus_quant": (I, [I, P, I64, I64, P, F, P, I, P, P, P]),
+            "orc_nvfp4_gptq": (I, [P, I64, I64, P, F, I, I, P, P, P, P, I]),
             "orc_scales_to_mma_layout": (None, [P, I64, I64, P]),
         }
         for name, (res, args) in sigs.items():
@@ -271,6 +272,29 @@ def mxfp4_dequant(codes: np.ndarray, scales: np.ndarray, rows: int, cols: int) -
     y = np.empty((rows, cols), dtype=np.float32)
     _load().orc_mxfp4_dequant(_ptr(codes), _ptr(scales), rows, cols, _ptr(y))
     return y
+
+
+def nvfp4_gptq(x: np.ndarray, U: np.ndarray, S=None, window=NVFP4_MSE_WINDOW, threads: int = 0) -> dict:
+    """ScaleSweep inside GPTQ (Cholesky form): `U` the upper Cholesky factor of
+    the inverse dampened Gram matrix (cols x cols, fp32; U^T U = H^-1).  S
+    defaults to the global scale of x.  Returns codes, scales, y and the scaled
+    errors err."""
+    x = _f32(x)
+    rows, cols = x.shape
+    U = _f32(U)
+    assert U.shape == (cols, cols)
+    if S is None:
+        S = global_scale(global_absmax(x))
+    codes = np.empty(rows * cols // 2, dtype=np.uint8)
+    scales = np.empty(rows * cols // NVFP4_BLOCK, dtype=np.uint8)
+    y = np.empty((rows, cols), dtype=np.float32)
+    err = np.empty((rows, cols), dtype=np.float32)
+    st = _load().orc_nvfp4_gptq(_ptr(x), rows, cols, _ptr(U), float(np.float32(S)), int(window[0]),
+                                int(window[1]), _ptr(codes), _ptr(scales), _ptr(y), _ptr(err), int(threads))
+    if st != STATUS_OK:
+        raise ValueError(f"oracle nvfp4_gptq failed with {st}")
+    return {"codes": codes.reshape(rows, cols // 2), "scales": scales.reshape(rows, cols // NVFP4_BLOCK),
+            "y": y, "err": err, "S": np.float32(S)}
 
 
 def hadamard32_inverse(y: np.ndarray, mask: int) -> np.ndarray:

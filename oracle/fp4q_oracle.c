@@ -42,6 +42,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #ifdef _OPENMP
@@ -256,6 +257,34 @@ static void pack_nibbles(const uint8_t* nib, int bs, uint8_t* out)
  * Outputs (each may be NULL): codes[rows*cols/2], scales[rows*cols/16],
  * y[rows*cols] (reconstruction in fp32), loss[rows*cols/16], base[...] (s_base
  * pattern). */
+/* The ScaleSweep selection for one 16-element block: s_base pattern p from
+ * amax / (6*S), then the window p+lo .. p+hi clipped to 0x01..0x7E, first
+ * minimum of block_loss.  Returns the chosen pattern; *best its loss, *base p. */
+static int sweep_select(const float* xb, const float* wb, float S, int lo, int hi, float* best, int* base)
+{
+    const int bs = 16;
+    float amax = 0.0f, t6, v;
+    int i, p, pp, first, last, bp = 0;
+    for (i = 0; i < bs; ++i) {
+        float a = fabsf(xb[i]);
+        if (a > amax) amax = a;
+    }
+    t6 = 6.0f * S;
+    v = amax / t6;
+    p = orc_e4m3_encode(v);
+    first = p + lo < 1 ? 1 : p + lo;
+    last = p + hi > 126 ? 126 : p + hi;
+    *best = 0.0f;
+    for (pp = first; pp <= last; ++pp) {
+        float d = orc_e4m3_value(pp) * S;
+        float inv = 1.0f / d;
+        float L = block_loss(xb, wb, bs, d, inv, NULL, NULL);
+        if (pp == first || L < *best) { *best = L; bp = pp; }
+    }
+    *base = p;
+    return bp;
+}
+
 int orc_nvfp4_quant(const float* x, int64_t rows, int64_t cols, float S,
                     const float* importance, int lo, int hi,
                     uint8_t* codes, uint8_t* scales, float* y, float* loss,
@@ -274,24 +303,10 @@ int orc_nvfp4_quant(const float* x, int64_t rows, int64_t cols, float S,
             const float* xb = x + r * cols + b * bs;
             const float* wb = importance ? importance + b * bs : NULL;
             int64_t blk = r * nb + b;
-            float amax = 0.0f, t6, v, best = 0.0f;
-            int i, p, pp, first, last, bp = 0;
+            float best = 0.0f;
+            int p, bp;
             uint8_t nib[16];
-            for (i = 0; i < bs; ++i) {
-                float a = fabsf(xb[i]);
-                if (a > amax) amax = a;
-            }
-            t6 = 6.0f * S;
-            v = amax / t6;
-            p = orc_e4m3_encode(v);
-            first = p + lo < 1 ? 1 : p + lo;
-            last = p + hi > 126 ? 126 : p + hi;
-            for (pp = first; pp <= last; ++pp) {
-                float d = orc_e4m3_value(pp) * S;
-                float inv = 1.0f / d;
-                float L = block_loss(xb, wb, bs, d, inv, NULL, NULL);
-                if (pp == first || L < best) { best = L; bp = pp; }
-            }
+            bp = sweep_select(xb, wb, S, lo, hi, &best, &p);
             {
                 float d = orc_e4m3_value(bp) * S;
                 float inv = 1.0f / d;
@@ -304,6 +319,71 @@ int orc_nvfp4_quant(const float* x, int64_t rows, int64_t cols, float S,
         }
     }
     return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* ScaleSweep inside GPTQ  ([SS] "Contribuicoes" 2)                          */
+/* ------------------------------------------------------------------------ */
+
+/* [SS] presents ScaleSweep as the block-scale selection of both RTN and GPTQ
+ * pipelines.  Reading (the page does not spell GPTQ out): GPTQ in its
+ * Cholesky form, with U the upper Cholesky factor of the inverse of the
+ * layer's dampened input Gram matrix (U^T U = H^-1), supplied by the caller.
+ * Rows are independent; along a row the columns are taken in order.  At the
+ * first column of every 16-column group the ScaleSweep (window lo..hi,
+ * global scale S of the original weight) picks the group's E4M3 pattern from
+ * the row's current, error-compensated values of the group; then every column
+ * j is quantized with its group's step d (inv = RN(1/d)) and its scaled error
+ * is spread over the later columns:
+ *   y_j = RN(E2M1(RN(w_j * inv)) * d);   e_j = RN((w_j - y_j) / U[j][j])
+ *   w_c = fma(-e_j, U[j][c], w_c)        for every c > j
+ * (each update one fused multiply-add, one rounding).  Outputs: codes,
+ * scales, the reconstruction y, and err[rows][cols] = e (may be NULL). */
+int orc_nvfp4_gptq(const float* x, int64_t rows, int64_t cols, const float* U, float S, int lo, int hi,
+                   uint8_t* codes, uint8_t* scales, float* y, float* err, int threads)
+{
+    const int bs = 16;
+    int64_t nb = cols / bs, r;
+    int status = ORC_OK;
+    if (cols % bs) return 2;
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(static)
+#endif
+    for (r = 0; r < rows; ++r) {
+        float* w = (float*)malloc((size_t)cols * sizeof(float));
+        int64_t j, c;
+        float d = 1.0f, inv = 1.0f;
+        uint8_t nib[16];
+        if (!w) {
+            status = 2;
+            continue;
+        }
+        for (j = 0; j < cols; ++j) w[j] = x[r * cols + j];
+        for (j = 0; j < cols; ++j) {
+            float rr, q, yy, e;
+            int code;
+            if (j % bs == 0) {
+                float best;
+                int base, bp = sweep_select(w + j, NULL, S, lo, hi, &best, &base);
+                d = orc_e4m3_value(bp) * S;
+                inv = 1.0f / d;
+                if (scales) scales[r * nb + j / bs] = (uint8_t)bp;
+            }
+            rr = w[j] * inv;
+            code = orc_e2m1_encode(rr);
+            q = orc_e2m1_decode(code);
+            yy = q * d;
+            e = (w[j] - yy) / U[j * cols + j];
+            nib[j % bs] = (uint8_t)code;
+            if (y) y[r * cols + j] = yy;
+            if (err) err[r * cols + j] = e;
+            for (c = j + 1; c < cols; ++c) w[c] = fmaf(-e, U[j * cols + c], w[c]);
+            if (j % bs == bs - 1 && codes) pack_nibbles(nib, bs, codes + (r * nb + j / bs) * (bs / 2));
+        }
+        free(w);
+    }
+    return status;
 }
 
 /* Exhaustive search statistics per block over all 126 finite positive E4M3
