@@ -551,6 +551,68 @@ def run_act_latency(args):
     return 0
 
 
+# --------------------------------------------------------------------------- GPTQ
+
+def run_gptq(args):
+    """Time fp4q_nvfp4_gptq (ScaleSweep inside GPTQ) on one synthetic weight
+    (`--shape`, default the WMSE workload's 11008 x 4096) with the Gram matrix
+    of 2048 synthetic bf16 activations (N(0,1), 1% of the columns x50).  Each
+    launch starts from a fresh fp32 copy of the weight (the call overwrites it;
+    the copy is inside the timed region, ~0.1 ms).  Reports the time and the
+    rate of the fused multiply-adds of the error updates (rows * cols^2 / 2)
+    against the FP32 lane peak.  Prints one JSON line (not the benchmark line)."""
+    import fp4_post_weight_grid_b200 as fq
+    from fp4_post_weight_grid_b200 import build as fbuild
+    import synth
+    fbuild.build()
+    rows, cols = (int(v) for v in args.shape.lower().split("x"))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w0 = synth.t_weight(rows, cols, nu=4, scale=0.02, seed=3, device=dev).float()
+    g = torch.Generator(device="cpu").manual_seed(3)
+    X = torch.randn(2048, cols, generator=g)
+    X[:, torch.randperm(cols, generator=g)[:max(1, cols // 100)]] *= 50.0
+    X = X.to(torch.bfloat16).to(dev, torch.float64)
+    H = X.T @ X
+    H += 0.01 * H.diagonal().mean() * torch.eye(cols, dtype=torch.float64, device=dev)
+    U = torch.linalg.cholesky(torch.cholesky_inverse(torch.linalg.cholesky(H))).mT.contiguous().float()
+    del X, H
+    w = torch.empty_like(w0)
+    amax = torch.empty(1, device=dev)
+    S = torch.empty(1, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+    deq = torch.empty_like(w0)
+    ws = torch.empty(fq.fp4q_gptq_workspace_bytes(rows), dtype=torch.uint8, device=dev)
+    fq.fp4q_global_absmax(w0, amax)
+    stream = torch.cuda.current_stream()
+
+    def launch():
+        w.copy_(w0)
+        fq.fp4q_nvfp4_gptq(w, U, amax, codes, scales, S, deq, ws, st, stream)
+
+    times = []
+    for i in range(max(args.warmup, 1) + args.steps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        launch()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= max(args.warmup, 1):
+            times.append(a.elapsed_time(b))
+    med = statistics.median(times)
+    fmas = rows * cols * (cols - 1) / 2
+    clk = load_peaks()[2]
+    peak = 148 * SM_FP32_LANES * clk * 1e6 / 1e12
+    print(json.dumps({"gptq": [rows, cols], "ms_median": med, "ms_min": min(times),
+                      "update_fma": fmas, "tfma_per_s": fmas / (med * 1e-3) / 1e12,
+                      "fp32_lane_peak_tfma_per_s": peak, "frac": fmas / (med * 1e-3) / 1e12 / peak,
+                      "status": int(st.item())}), flush=True)
+    return 0
+
+
 # --------------------------------------------------------------------------- main
 
 def main():
@@ -561,6 +623,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gptq", action="store_true",
+                    help="time the ScaleSweep inside GPTQ on one weight (default 11008x4096)")
     ap.add_argument("--act-latency", action="store_true",
                     help="per-call latency of the NVFP4 sweep on activation-sized tensors, two calls vs one launch")
     ap.add_argument("--single", choices=sorted(SINGLE_PATHS), default=None,
@@ -582,6 +646,10 @@ def main():
         return run_single(args)
     if args.act_latency:
         return run_act_latency(args)
+    if args.gptq:
+        if args.shape == "16384x8192":
+            args.shape = "11008x4096"
+        return run_gptq(args)
 
     import fp4_post_weight_grid_b200 as fq
     from fp4_post_weight_grid_b200 import build as fbuild

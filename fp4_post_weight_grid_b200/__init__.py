@@ -30,6 +30,7 @@ __all__ = [
     "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes", "nvfp4_quantize_dynamic",
     "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout", "mma_scales",
     "fp4q_focus_quant", "fp4q_mxfp4_unrotate", "focus_quantize", "mxfp4_unrotate", "FocusResult",
+    "fp4q_nvfp4_gptq", "fp4q_gptq_workspace_bytes", "nvfp4_gptq",
     "quantize_batch",
     "NVFP4Result", "MXFP4Result", "nvfp4_quantize", "mxfp4_quantize", "quantize_dual", "dequantize",
     "FLAG_NONFINITE", "FLAG_RANGE", "FLAG_TIMEOUT",
@@ -50,7 +51,8 @@ EXPORTS = ("fp4q_version", "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_g
            "fp4q_mxfp4_quant_hadamard", "fp4q_mxfp4_quant_absmax", "fp4q_quantize_dual",
            "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_quantize_batch_static", "fp4q_dequant",
            "fp4q_probe_e2m1", "fp4q_probe_e4m3", "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes",
-           "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout", "fp4q_focus_quant", "fp4q_mxfp4_unrotate")
+           "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout", "fp4q_focus_quant", "fp4q_mxfp4_unrotate",
+           "fp4q_nvfp4_gptq", "fp4q_gptq_workspace_bytes")
 
 
 class BatchTensor(ctypes.Structure):
@@ -111,6 +113,7 @@ def load():
     sigs["fp4q_scales_to_mma_layout"] = [P, I64, I64, P, P]
     sigs["fp4q_focus_quant"] = [I, P, I, I64, I64, P, P, P, ctypes.c_int32, P, P, P, P, P]
     sigs["fp4q_mxfp4_unrotate"] = [P, I, I64, I64, P, P, P]
+    sigs["fp4q_nvfp4_gptq"] = [P, I64, I64, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]
     sigs["fp4q_nvfp4_sweep_dynamic"] = [P, I, I64, I64, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -118,6 +121,8 @@ def load():
         fn.argtypes = args
     lib.fp4q_batch_workspace_bytes.restype = ctypes.c_size_t
     lib.fp4q_batch_workspace_bytes.argtypes = []
+    lib.fp4q_gptq_workspace_bytes.restype = ctypes.c_size_t
+    lib.fp4q_gptq_workspace_bytes.argtypes = [I64]
     lib.fp4q_mma_scale_bytes.restype = I64
     lib.fp4q_mma_scale_bytes.argtypes = [I64, I64]
     lib.fp4q_dynamic_workspace_bytes.restype = ctypes.c_size_t
@@ -300,6 +305,30 @@ def fp4q_mxfp4_unrotate(y, sign_masks, out, stream=None) -> None:
                                       _dev(sign_masks, "sign_masks", (torch.int32, torch.uint32), cols // 32, dev),
                                       _dev(out, "out", y.dtype, rows * cols, dev), _stream(stream)),
            "fp4q_mxfp4_unrotate")
+
+
+def fp4q_gptq_workspace_bytes(rows: int) -> int:
+    return int(load().fp4q_gptq_workspace_bytes(int(rows)))
+
+
+def fp4q_nvfp4_gptq(w, U, d_amax, codes, scales, d_global_scale, deq, workspace, d_status, stream=None) -> None:
+    """ScaleSweep inside GPTQ.  `w` (float32, contiguous) is overwritten with
+    the error-compensated values; `U` the upper Cholesky factor of H^-1."""
+    rows, cols = _rc(w, NVFP4_BLOCK)
+    if w.dtype != torch.float32:
+        raise TypeError("fp4q_nvfp4_gptq works on a float32 copy of the weight")
+    dev = w.device
+    n = rows * cols
+    ws = _dev(workspace, "workspace", device=dev)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load().fp4q_nvfp4_gptq(_dev(w, "w", device=dev), rows, cols, _dev(U, "U", torch.float32, cols * cols, dev),
+                                  _dev(d_amax, "d_amax", torch.float32, 1, dev),
+                                  _dev(codes, "codes", torch.uint8, n // 2, dev),
+                                  _dev(scales, "scales", torch.uint8, n // NVFP4_BLOCK, dev),
+                                  _dev(d_global_scale, "d_global_scale", torch.float32, 1, dev),
+                                  _dev(deq, "deq", torch.float32, n, dev), ws, nbytes,
+                                  _dev(d_status, "d_status", torch.int32, 1, dev), _stream(stream)),
+           "fp4q_nvfp4_gptq")
 
 
 def fp4q_mma_scale_bytes(rows: int, scale_cols: int) -> int:
@@ -537,6 +566,24 @@ def focus_quantize(w: torch.Tensor, fmt: int, scales: torch.Tensor, coeffs: torc
     status = torch.zeros(1, dtype=torch.int32, **kw)
     fp4q_focus_quant(fmt, w, scales, global_scale, coeffs, sub_block, codes, deq, loss, status, stream)
     return FocusResult(codes, deq, loss, status)
+
+
+def nvfp4_gptq(w: torch.Tensor, U: torch.Tensor, with_deq=True, stream=None) -> NVFP4Result:
+    """Allocating form of fp4q_nvfp4_gptq on a float32 copy of `w` (the input is
+    not modified); the global scale is that of `w`."""
+    rows, cols = _rc(w, NVFP4_BLOCK)
+    kw = dict(device=w.device)
+    work = w.to(torch.float32).contiguous().clone()
+    amax = torch.empty(1, dtype=torch.float32, **kw)
+    fp4q_global_absmax(work, amax, stream)
+    S = torch.empty(1, dtype=torch.float32, **kw)
+    status = torch.zeros(1, dtype=torch.int32, **kw)
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, **kw)
+    scales = torch.empty((rows, cols // NVFP4_BLOCK), dtype=torch.uint8, **kw)
+    deq = torch.empty((rows, cols), dtype=torch.float32, **kw) if with_deq else None
+    ws = torch.empty(max(fp4q_gptq_workspace_bytes(rows), 16), dtype=torch.uint8, **kw)
+    fp4q_nvfp4_gptq(work, U, amax, codes, scales, S, deq, ws, status, stream)
+    return NVFP4Result(codes, scales, S, deq, None, amax, status)
 
 
 def mxfp4_unrotate(y: torch.Tensor, sign_masks: torch.Tensor, stream=None) -> torch.Tensor:

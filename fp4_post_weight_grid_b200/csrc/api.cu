@@ -269,6 +269,35 @@ fp4q_status fp4q_mxfp4_unrotate(const void* y, fp4q_dtype dt, int64_t rows, int6
     return after_launch();
 }
 
+size_t fp4q_gptq_workspace_bytes(int64_t rows)
+{
+    return rows > 0 ? fp4q::gptq_workspace_bytes(rows) : 0;
+}
+
+fp4q_status fp4q_nvfp4_gptq(float* w, int64_t rows, int64_t cols, const float* U, const float* d_amax,
+                            uint8_t* codes, uint8_t* scales_e4m3, float* d_global_scale, float* deq,
+                            void* workspace, size_t workspace_bytes, int32_t* d_status, fp4q_stream_t stream)
+{
+    bool empty = false;
+    fp4q_status st = check_quant_args(w, FP4Q_F32, rows, cols, FP4Q_NVFP4_BLOCK, codes, scales_e4m3, d_status,
+                                      deq, nullptr, 8, &empty);
+    if (st != FP4Q_OK || empty) return st;
+    if (cols > (int64_t)1 << 20) return FP4Q_ERR_SHAPE;        // U alone would be 4 TB
+    if (!U || !d_amax || !d_global_scale || !workspace) return FP4Q_ERR_NULL;
+    if (!aligned(U, 4) || !aligned(d_amax, 4) || !aligned(d_global_scale, 4) || !aligned(workspace, 16))
+        return FP4Q_ERR_ALIGN;
+    if (workspace_bytes < fp4q_gptq_workspace_bytes(rows)) return FP4Q_ERR_ARG;
+    const cudaError_t e = fp4q::launch_nvfp4_gptq(w, rows, cols, U, d_amax, codes, scales_e4m3, d_global_scale, deq,
+                                                  static_cast<float*>(workspace), d_status,
+                                                  reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        std::strncpy(g_last_cuda_error, cudaGetErrorString(e), sizeof(g_last_cuda_error) - 1);
+        g_last_cuda_error[sizeof(g_last_cuda_error) - 1] = '\0';
+        return FP4Q_ERR_CUDA;
+    }
+    return FP4Q_OK;
+}
+
 int64_t fp4q_mma_scale_bytes(int64_t rows, int64_t scale_cols)
 {
     if (rows < 0 || scale_cols < 0 || (scale_cols != 0 && rows > INT64_MAX / 1024 / scale_cols)) return -1;

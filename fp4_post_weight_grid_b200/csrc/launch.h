@@ -59,6 +59,13 @@ bool launch_focus(bool mx, bool bf16, int sub, const void* w, int64_t rows, int6
 void launch_unrotate(bool bf16, const void* y, int64_t rows, int64_t cols, const uint32_t* sign_masks, void* out,
                      cudaStream_t s);
 
+// ScaleSweep inside GPTQ: w (fp32, rows x cols) is updated in place; E is the
+// workspace of gptq_workspace_bytes(rows) bytes.
+size_t gptq_workspace_bytes(int64_t rows);
+cudaError_t launch_nvfp4_gptq(float* w, int64_t rows, int64_t cols, const float* U, const float* d_amax,
+                              uint8_t* codes, uint8_t* scales, float* d_S, float* deq, float* E, int32_t* d_status,
+                              cudaStream_t s);
+
 // Block scales [rows][scols] -> the 128 x 4 tiled layout of block-scaled GEMMs.
 int64_t mma_scale_bytes(int64_t rows, int64_t scols);
 void launch_mma_scale_layout(const uint8_t* s, int64_t rows, int64_t scols, uint8_t* out, cudaStream_t st);

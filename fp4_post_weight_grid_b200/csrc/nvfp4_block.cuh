@@ -66,74 +66,35 @@ __device__ __forceinline__ NvScale nvfp4_scale(float gmax)
 }
 
 // Fill the tables for global scale S.  Every thread of the thread block must
-// call it (it synchronises twice); blockDim.x >= kNvPairs.
+// call it (it synchronises twice); any block size.
 __device__ __forceinline__ void nvfp4_tables(NvTables& t, float S)
 {
-    if (threadIdx.x < 128) {
-        const uint32_t p = threadIdx.x == 0 ? 1u : (threadIdx.x == 127 ? 126u : threadIdx.x);
+    for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+        const uint32_t p = i == 0 ? 1u : (i == 127 ? 126u : (uint32_t)i);
         const float v = e4m3_value(p);
         const float d = __fmul_rn(v, S);
-        t.step[threadIdx.x] = make_float4(d, __frcp_rn(d), __fmul_rn(v, v), 0.0f);
+        t.step[i] = make_float4(d, __frcp_rn(d), __fmul_rn(v, v), 0.0f);
     }
     __syncthreads();
-    if (threadIdx.x < kNvPairs) {
-        const int pa = min(max((int)threadIdx.x - kNvOff, 1), 126);
-        const int pb = min(max((int)threadIdx.x - kNvOff + 1, 1), 126);
-        t.inv_pair[threadIdx.x] = make_float2(t.step[pa].y, t.step[pb].y);
-        t.vsq_pair[threadIdx.x] = make_float2(t.step[pa].z, t.step[pb].z);
+    for (int i = threadIdx.x; i < kNvPairs; i += blockDim.x) {
+        const int pa = min(max(i - kNvOff, 1), 126);
+        const int pb = min(max(i - kNvOff + 1, 1), 126);
+        t.inv_pair[i] = make_float2(t.step[pa].y, t.step[pb].y);
+        t.vsq_pair[i] = make_float2(t.step[pa].z, t.step[pb].z);
     }
     __syncthreads();
 }
 
-// Quantize one 16-element block.
-//   src        the block's 16 input elements
-//   wimp       the block's 16 importance weights (WMSE only)
-//   codes8     8 bytes of packed nibbles; scale: the E4M3 pattern byte
-//   deq16      16 reconstructed elements or nullptr; loss: the block's loss or nullptr
-template <typename T, int LO, int NREAL, bool WMSE>
-__device__ __forceinline__ void nvfp4_block(const NvTables& tb, const NvScale& c, const T* __restrict__ src,
-                                            const float* __restrict__ wimp, uint8_t* __restrict__ codes8,
-                                            uint8_t* __restrict__ scale, T* __restrict__ deq16,
-                                            float* __restrict__ loss, uint64_t z2, float neg_zero)
+// Choose the pattern of one block: the screen, the survivor threshold and the
+// exact verification below, on the block's 16 values x (amax = max|x|;
+// wt the importance weights for WMSE; alpha2, tau and prune as in
+// screen.cuh).  Returns the winning E4M3 pattern.
+template <int LO, int NREAL, bool WMSE>
+__device__ __forceinline__ int nvfp4_select(const NvTables& tb, const NvScale& c, const float (&x)[16], float amax,
+                                            const float (&wt)[16], float alpha2, float tau, bool prune,
+                                            uint64_t z2, float neg_zero)
 {
     constexpr int NC = (NREAL + 1) & ~1;
-    // The search works on the signed values: E2M1 rounding and every loss
-    // term are symmetric in the sign, so the losses equal those of |x|.
-    float x[16];
-    uint32_t abits;
-    load_block_amax<16>(src, x, abits);
-    const float amax = __uint_as_float(abits);
-    float alpha2;
-    float wt[16];
-    float tau = c.tau0;
-    bool prune = true;
-    if (WMSE) {
-        const float4* wp = reinterpret_cast<const float4*>(wimp);
-        uint32_t wbits = 0;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            const float4 t = __ldg(wp + v);
-            wt[4 * v + 0] = t.x; wt[4 * v + 1] = t.y; wt[4 * v + 2] = t.z; wt[4 * v + 3] = t.w;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) wbits = max(wbits, __float_as_uint(wt[i]));
-        // the bound assumes 0 <= w <= 2^64 (sign bit clear, at most 2^64)
-        prune = wbits <= 0x5F800000u;
-        tau = c.tau0 * (1.0f + __uint_as_float(min(wbits, 0x5F800000u)));
-        uint64_t al2 = pk(0.0f, 0.0f);
-        const uint64_t invS2 = pk(c.invS, c.invS);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint64_t xs = mul2(pk(x[2 * j], x[2 * j + 1]), invS2);
-            al2 = fma2(mul2(pk(wt[2 * j], wt[2 * j + 1]), xs), xs, al2);
-        }
-        float lo, hi;
-        upk(al2, lo, hi);
-        alpha2 = (lo + hi) * (1.0f + 0x1p-16f);   // bound only: rounded up generously
-    } else {
-        const float as = amax * c.invS;            // sum x^2 / S^2 <= 16 amax^2 / S^2
-        alpha2 = (16.0f * as * as) * (1.0f + 0x1p-16f);
-    }
     const int p = (int)e4m3_rn_sat(__fdiv_rn(amax, c.t6));   // s_base pattern
 
     // 1. screen every candidate of the window
@@ -220,6 +181,59 @@ __device__ __forceinline__ void nvfp4_block(const NvTables& tb, const NvScale& c
             first = false;
         }
     }
+
+    return bp;
+}
+
+// Quantize one 16-element block.
+//   src        the block's 16 input elements
+//   wimp       the block's 16 importance weights (WMSE only)
+//   codes8     8 bytes of packed nibbles; scale: the E4M3 pattern byte
+//   deq16      16 reconstructed elements or nullptr; loss: the block's loss or nullptr
+template <typename T, int LO, int NREAL, bool WMSE>
+__device__ __forceinline__ void nvfp4_block(const NvTables& tb, const NvScale& c, const T* __restrict__ src,
+                                            const float* __restrict__ wimp, uint8_t* __restrict__ codes8,
+                                            uint8_t* __restrict__ scale, T* __restrict__ deq16,
+                                            float* __restrict__ loss, uint64_t z2, float neg_zero)
+{
+    // The search works on the signed values: E2M1 rounding and every loss
+    // term are symmetric in the sign, so the losses equal those of |x|.
+    float x[16];
+    uint32_t abits;
+    load_block_amax<16>(src, x, abits);
+    const float amax = __uint_as_float(abits);
+    float alpha2;
+    float wt[16];
+    float tau = c.tau0;
+    bool prune = true;
+    if (WMSE) {
+        const float4* wp = reinterpret_cast<const float4*>(wimp);
+        uint32_t wbits = 0;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const float4 t = __ldg(wp + v);
+            wt[4 * v + 0] = t.x; wt[4 * v + 1] = t.y; wt[4 * v + 2] = t.z; wt[4 * v + 3] = t.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) wbits = max(wbits, __float_as_uint(wt[i]));
+        // the bound assumes 0 <= w <= 2^64 (sign bit clear, at most 2^64)
+        prune = wbits <= 0x5F800000u;
+        tau = c.tau0 * (1.0f + __uint_as_float(min(wbits, 0x5F800000u)));
+        uint64_t al2 = pk(0.0f, 0.0f);
+        const uint64_t invS2 = pk(c.invS, c.invS);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint64_t xs = mul2(pk(x[2 * j], x[2 * j + 1]), invS2);
+            al2 = fma2(mul2(pk(wt[2 * j], wt[2 * j + 1]), xs), xs, al2);
+        }
+        float lo, hi;
+        upk(al2, lo, hi);
+        alpha2 = (lo + hi) * (1.0f + 0x1p-16f);   // bound only: rounded up generously
+    } else {
+        const float as = amax * c.invS;            // sum x^2 / S^2 <= 16 amax^2 / S^2
+        alpha2 = (16.0f * as * as) * (1.0f + 0x1p-16f);
+    }
+    const int bp = nvfp4_select<LO, NREAL, WMSE>(tb, c, x, amax, wt, alpha2, tau, prune, z2, neg_zero);
 
     // 3. emit the winner: codes from the signed values, reconstruction q*d,
     //    and its exact loss when requested

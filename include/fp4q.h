@@ -279,6 +279,41 @@ fp4q_status fp4q_mxfp4_unrotate(const void* y, fp4q_dtype dt, int64_t rows, int6
                                 const uint32_t* sign_masks, void* out, fp4q_stream_t stream);
 
 /*
+ * fp4q_gptq_workspace_bytes -- workspace of fp4q_nvfp4_gptq: rows * 128 floats.
+ */
+size_t fp4q_gptq_workspace_bytes(int64_t rows);
+
+/*
+ * fp4q_nvfp4_gptq -- NVFP4 with the ScaleSweep inside GPTQ (ScaleSweep
+ * summary, "Contribuicoes" 2: the sweep selects the block scales of GPTQ
+ * pipelines too).  GPTQ in its Cholesky form: U is the upper Cholesky factor
+ * of the inverse of the layer's dampened input Gram matrix (U^T U = H^-1;
+ * the caller computes it).  Rows are independent; along a row, at the first
+ * column of every 16-column group the ScaleSweep (MSE window -3..+7, global
+ * scale S = max|w|/1536 of the ORIGINAL weight) picks the group's pattern from
+ * the row's current, error-compensated values, and every column j is
+ * quantized with its group's step d and spreads its error:
+ *   y_j = RN(E2M1(RN(w_j * RN(1/d))) * d);   e_j = RN((w_j - y_j) / U[j][j])
+ *   w_c = fma(-e_j, U[j][c], w_c) for every c > j (one rounding each).
+ * The blocked GPU algorithm applies these updates to every element in the
+ * same order, so its bytes are those of the sequential definition.
+ *   w          device fp32 rows x cols (cols % 16 == 0), 16-byte aligned;
+ *              OVERWRITTEN with the error-compensated values.
+ *   U          device fp32 cols x cols, row-major; only the upper triangle
+ *              (diagonal included) is read.
+ *   d_amax     device float: max|w| of the original weight
+ *              (fp4q_global_absmax before this call).
+ *   codes, scales_e4m3, d_global_scale, deq (fp32, may be NULL) as
+ *              fp4q_nvfp4_sweepmse.
+ *   workspace  device, 16-byte aligned, fp4q_gptq_workspace_bytes(rows).
+ * 2 * ceil(cols/128) launches.  Errors as fp4q_nvfp4_sweepmse, plus
+ * FP4Q_ERR_ARG for a small workspace and FP4Q_ERR_SHAPE for cols > 2^20.
+ */
+fp4q_status fp4q_nvfp4_gptq(float* w, int64_t rows, int64_t cols, const float* U, const float* d_amax,
+                            uint8_t* codes, uint8_t* scales_e4m3, float* d_global_scale, float* deq,
+                            void* workspace, size_t workspace_bytes, int32_t* d_status, fp4q_stream_t stream);
+
+/*
  * fp4q_mma_scale_bytes -- bytes of the tiled scale layout written by
  * fp4q_scales_to_mma_layout for a [rows][scale_cols] scale matrix:
  * ceil(rows/128) * ceil(scale_cols/4) * 512; -1 for a negative or
