@@ -15,15 +15,17 @@
 // in ascending j, whether they are applied column by column or block by
 // block; so the blocked algorithm below writes exactly the bytes of the plain
 // sequential one.  Per block of 128 columns:
-//   gptq_block_kernel   one thread per row (64 rows per thread block): the
-//                       block's slice of each row and U's diagonal block in
-//                       shared memory; the sweep at every group start, the
-//                       column quantization, the error and the in-block
-//                       updates; the scaled errors go to a workspace E;
-//   gptq_update_kernel  the trailing update w[:, c] for the columns after the
-//                       block, a 64 x 64 output tile per thread block, each
-//                       output a chain of exact fused multiply-adds over the
-//                       block's 128 columns in ascending order.
+//   gptq_block_kernel   8 threads per row, each holding one 16-column group
+//                       of the block in registers, U's diagonal block in
+//                       shared memory: the sweep at every group start, the
+//                       column quantization by the group's owner, the error
+//                       broadcast by a warp shuffle, the in-block updates;
+//                       the scaled errors go to a workspace E;
+//   gptq_update_kernel  the trailing update of the columns after the block,
+//                       a 128 x 128 output tile per thread block (8 x 8 per
+//                       thread), each output a chain of exact fused
+//                       multiply-adds over the block's columns in ascending
+//                       order.
 // The trailing update is a dense contraction, but it runs on the CUDA cores:
 // its definition is a chain of single-rounding fused multiply-adds in a fixed
 // order, which a tensor-core accumulation (another precision and order) would
@@ -37,20 +39,25 @@ namespace fp4q {
 namespace {
 
 constexpr int kB = 128;           // columns per block
-constexpr int kRowsA = 64;        // rows (threads) per thread block of the inner kernel
-constexpr int kTile = 64;         // output tile of the update kernel (rows and columns)
+constexpr int kLanes = 8;         // threads per row in the in-block kernel: one 16-column group each
+constexpr int kThreadsA = 256;    // 32 rows per thread block
+constexpr int kTB = 128;          // output tile of the update kernel (rows and columns)
+constexpr int kBK = 32;           // block columns per shared-memory chunk of the update kernel
 
-__global__ void __launch_bounds__(kRowsA)
+// In-block GPTQ.  Thread `lane` of a row keeps the row's 16 values of group
+// `lane` of the block in registers.  For every column j of group g, the owner
+// (lane g) quantizes it (after the ScaleSweep of the group at its first
+// column), computes e_j and broadcasts it to the row's other lanes with a
+// warp shuffle; every lane then updates its own later columns with
+// w_c = fma(-e_j, U[j][c], w_c), so each value sees the updates in ascending j.
+__global__ void __launch_bounds__(kThreadsA)
 gptq_block_kernel(const float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0, int bw,
                   const float* __restrict__ U, const float* __restrict__ d_amax, uint8_t* __restrict__ codes,
                   uint8_t* __restrict__ scales, float* __restrict__ d_S, float* __restrict__ deq,
-                  float* __restrict__ E, int32_t* __restrict__ d_status, float neg_zero)
+                  float* __restrict__ Et, int64_t ldE, int32_t* __restrict__ d_status, float neg_zero)
 {
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float Us[];      // [bw][bw]: U's diagonal block
     __shared__ NvTables tb;
-    const int ld = bw + 1;                           // padded row stride: no bank conflicts
-    float* Ws = sm;                                  // [kRowsA][ld]
-    float* Us = sm + kRowsA * ld;                    // [bw][bw]
     const float gmax = __ldg(d_amax);
     const int32_t flag = nvfp4_gmax_flag(gmax);
     if (flag) {
@@ -59,132 +66,206 @@ gptq_block_kernel(const float* __restrict__ w, int64_t rows, int64_t cols, int64
     }
     const NvScale c = nvfp4_scale(gmax);
     if (blockIdx.x == 0 && threadIdx.x == 0 && j0 == 0) *d_S = c.S;
-    const int64_t r0 = (int64_t)blockIdx.x * kRowsA;
-    for (int i = threadIdx.x; i < bw * bw; i += kRowsA)
+    for (int i = threadIdx.x; i < bw * bw; i += kThreadsA)
         Us[i] = __ldg(U + (j0 + i / bw) * cols + j0 + i % bw);
-    for (int i = threadIdx.x; i < kRowsA * bw; i += kRowsA) {
-        const int rr = i / bw, k = i % bw;
-        Ws[rr * ld + k] = r0 + rr < rows ? w[(r0 + rr) * cols + j0 + k] : 0.0f;
-    }
-    nvfp4_tables(tb, c.S);                           // synchronises: the slices are in place too
+    nvfp4_tables(tb, c.S);                           // synchronises: U's block is in place too
 
-    const int64_t row = r0 + threadIdx.x;
+    const int lane = threadIdx.x & (kLanes - 1);
+    const int src0 = (threadIdx.x & 31) & ~(kLanes - 1);   // this row's first lane in the warp
+    const int64_t row = (int64_t)blockIdx.x * (kThreadsA / kLanes) + threadIdx.x / kLanes;
+    const int ngroups = bw / 16;
     const bool active = row < rows;
-    float* wr = Ws + threadIdx.x * ld;
+    const bool mine = active && lane < ngroups;
+    float x[16];
+    if (mine) {
+        const float4* p = reinterpret_cast<const float4*>(w + row * cols + j0 + 16 * lane);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const float4 t = p[v];
+            x[4 * v + 0] = t.x; x[4 * v + 1] = t.y; x[4 * v + 2] = t.z; x[4 * v + 3] = t.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[k] = 0.0f;
+    }
     const uint64_t z2 = pk(neg_zero, neg_zero);
-    float d = 1.0f, inv = 1.0f;
-    uint64_t nib = 0;
 #pragma unroll 1
-    for (int j = 0; j < bw; ++j) {
-        if ((j & 15) == 0) {                         // the ScaleSweep of the group's current values
-            float x[16], wt[16];
+    for (int g = 0; g < ngroups; ++g) {
+        float d = 1.0f, inv = 1.0f;
+        if (lane == g) {                             // the ScaleSweep of the group's current values
+            float wt[16];
             float amax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                x[i] = wr[j + i];
-                amax = fmaxf(amax, fabsf(x[i]));
-            }
+            for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[k]));
             const float as = amax * c.invS;
             const float alpha2 = (16.0f * as * as) * (1.0f + 0x1p-16f);
             const int bp = nvfp4_select<-3, 11, false>(tb, c, x, amax, wt, alpha2, c.tau0, true, z2, neg_zero);
             const float4 st = tb.step[bp];
             d = st.x;
             inv = st.y;
-            if (active) scales[row * (cols / 16) + (j0 + j) / 16] = (uint8_t)bp;
-            nib = 0;
+            if (active) scales[row * (cols / 16) + (j0 + 16 * g) / 16] = (uint8_t)bp;
         }
-        const float wj = wr[j];
-        const uint32_t code = e2m1x2(__fmul_rn(wj, inv), 0.0f) & 0xFu;
-        float q, unused;
-        f16x2_to_f32(e2m1x2_to_f16x2(code), q, unused);
-        const float y = __fmul_rn(q, d);
-        const float e = __fdiv_rn(__fsub_rn(wj, y), Us[j * bw + j]);
-        nib |= (uint64_t)code << (4 * (j & 15));
-        if (active) {
-            E[row * kB + j] = e;
-            if (deq) deq[row * cols + j0 + j] = y;
-            if ((j & 15) == 15) *reinterpret_cast<uint64_t*>(codes + (row * cols + j0 + j - 15) / 2) = nib;
+        uint64_t nib = 0;
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+            const int j = 16 * g + jj;
+            float e = 0.0f;
+            if (lane == g) {
+                const float wj = x[jj];
+                const uint32_t code = e2m1x2(__fmul_rn(wj, inv), 0.0f) & 0xFu;
+                float q, unused;
+                f16x2_to_f32(e2m1x2_to_f16x2(code), q, unused);
+                const float y = __fmul_rn(q, d);
+                e = __fdiv_rn(__fsub_rn(wj, y), Us[j * bw + j]);
+                nib |= (uint64_t)code << (4 * jj);
+                if (active) {
+                    Et[j * ldE + row] = e;
+                    if (deq) deq[row * cols + j0 + j] = y;
+                }
+            }
+            e = __shfl_sync(0xFFFFFFFFu, e, src0 + g);
+            const float4* u4 = reinterpret_cast<const float4*>(Us + j * bw + 16 * lane);
+            if (lane > g && lane < ngroups) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const float4 u = u4[v];
+                    x[4 * v + 0] = __fmaf_rn(-e, u.x, x[4 * v + 0]);
+                    x[4 * v + 1] = __fmaf_rn(-e, u.y, x[4 * v + 1]);
+                    x[4 * v + 2] = __fmaf_rn(-e, u.z, x[4 * v + 2]);
+                    x[4 * v + 3] = __fmaf_rn(-e, u.w, x[4 * v + 3]);
+                }
+            } else if (lane == g) {
+                const float* uj = Us + j * bw + 16 * g;
+#pragma unroll
+                for (int k = jj + 1; k < 16; ++k) x[k] = __fmaf_rn(-e, uj[k], x[k]);
+            }
         }
-        const float* uj = Us + j * bw;
-#pragma unroll 4
-        for (int k = j + 1; k < bw; ++k) wr[k] = __fmaf_rn(-e, uj[k], wr[k]);
+        if (lane == g && active)
+            *reinterpret_cast<uint64_t*>(codes + (row * cols + j0 + 16 * g) / 2) = nib;
     }
 }
 
-__global__ void __launch_bounds__(256)
-gptq_update_kernel(float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0, int bw,
-                   const float* __restrict__ U, const float* __restrict__ E)
+// Trailing update w[r][c] for the columns after the block: a 128 x 128 output
+// tile per thread block, 8 x 8 outputs per thread (rows tr..tr+3, tr+64..tr+67
+// and columns tc..tc+3, tc+64..tc+67).  The block's columns are taken in
+// chunks of 32, in ascending order, through two shared-memory buffers filled
+// by asynchronous copies (the next chunk loads while this one is used); each
+// output is a chain of fused multiply-adds in ascending k.  Padding (rows or
+// columns past the end, k past the block) is zero-filled, and fma(-0, 0, a)
+// returns a unchanged.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid)
 {
-    extern __shared__ float sm[];
-    float* Es = sm;                                  // [bw][kTile]: E transposed, this tile's rows
-    float* Ut = sm + bw * kTile;                     // [bw][kTile]: U rows of the block, this tile's columns
-    const int64_t c_begin = j0 + bw;
-    const int64_t r0 = (int64_t)blockIdx.x * kTile;
-    const int64_t c0 = c_begin + (int64_t)blockIdx.y * kTile;
-    for (int i = threadIdx.x; i < bw * kTile; i += 256) {
-        const int k = i / kTile, t = i % kTile;      // coalesced along t for U, strided for E
-        Ut[i] = c0 + t < cols ? __ldg(U + (j0 + k) * cols + c0 + t) : 0.0f;
+    const unsigned dst = (unsigned)__cvta_generic_to_shared(smem);
+    const int n = valid ? 16 : 0;                   // 0: no bytes read, 16 zero bytes written
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(gmem), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ void gptq_load_chunk(float* Es, float* Ut, const float* __restrict__ Et, int64_t ldE,
+                                                const float* __restrict__ U, int64_t rows, int64_t cols, int64_t j0,
+                                                int bw, int kc, int64_t r0, int64_t c0)
+{
+    // 32 x 128 floats each, 16 bytes per copy: 4 copies of each per thread
+#pragma unroll
+    for (int s = 0; s < kBK * kTB / 4 / 256; ++s) {
+        const int i = threadIdx.x + 256 * s;
+        const int k = i / (kTB / 4), t = (i % (kTB / 4)) * 4;
+        const bool kin = kc + k < bw;
+        const bool ein = kin && r0 + t < rows;       // ldE is a multiple of 4: a 4-row group is all in or all out
+        const bool uin = kin && c0 + t < cols;       // cols is a multiple of 16
+        cp_async16(Es + k * kTB + t, ein ? Et + (int64_t)(kc + k) * ldE + r0 + t : Et, ein);
+        cp_async16(Ut + k * kTB + t, uin ? U + (j0 + kc + k) * cols + c0 + t : U, uin);
     }
-    for (int i = threadIdx.x; i < bw * kTile; i += 256) {
-        const int t = i / bw, k = i % bw;            // coalesced along k for E
-        Es[k * kTile + t] = r0 + t < rows ? __ldg(E + (r0 + t) * kB + k) : 0.0f;
-    }
-    __syncthreads();
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(256, 2)
+gptq_update_kernel(float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0, int bw,
+                   const float* __restrict__ U, const float* __restrict__ Et, int64_t ldE)
+{
+    extern __shared__ __align__(16) float sm[];      // 2 x {E chunk [k][row], U chunk [k][column]}
+    const int64_t r0 = (int64_t)blockIdx.x * kTB;
+    const int64_t c0 = j0 + bw + (int64_t)blockIdx.y * kTB;
     const int tr = (threadIdx.x >> 4) * 4, tc = (threadIdx.x & 15) * 4;
-    float acc[4][4];
+    const int nchunks = (bw + kBK - 1) / kBK;
+    gptq_load_chunk(sm, sm + kBK * kTB, Et, ldE, U, rows, cols, j0, bw, 0, r0, c0);
+    float acc[8][8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i) {
+        const int64_t r = r0 + tr + (i & 3) + (i >> 2) * 64;
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const int64_t r = r0 + tr + i, cc = c0 + tc + jj;
+        for (int jj = 0; jj < 8; ++jj) {
+            const int64_t cc = c0 + tc + (jj & 3) + (jj >> 2) * 64;
             acc[i][jj] = (r < rows && cc < cols) ? w[r * cols + cc] : 0.0f;
         }
-#pragma unroll 4
-    for (int k = 0; k < bw; ++k) {
-        const float4 a = *reinterpret_cast<const float4*>(Es + k * kTile + tr);
-        const float4 b = *reinterpret_cast<const float4*>(Ut + k * kTile + tc);
-        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+    }
+    for (int ch = 0; ch < nchunks; ++ch) {
+        float* Es = sm + (ch & 1) * 2 * kBK * kTB;
+        float* Ut = Es + kBK * kTB;
+        if (ch + 1 < nchunks) {
+            float* En = sm + ((ch + 1) & 1) * 2 * kBK * kTB;
+            gptq_load_chunk(En, En + kBK * kTB, Et, ldE, U, rows, cols, j0, bw, (ch + 1) * kBK, r0, c0);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();                             // chunk ch is in shared memory for every thread
+#pragma unroll 2
+        for (int k = 0; k < kBK; ++k) {
+            const float4 a0 = *reinterpret_cast<const float4*>(Es + k * kTB + tr);
+            const float4 a1 = *reinterpret_cast<const float4*>(Es + k * kTB + tr + 64);
+            const float4 b0 = *reinterpret_cast<const float4*>(Ut + k * kTB + tc);
+            const float4 b1 = *reinterpret_cast<const float4*>(Ut + k * kTB + tc + 64);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) acc[i][jj] = __fmaf_rn(-av[i], bv[jj], acc[i][jj]);
+                for (int jj = 0; jj < 8; ++jj) acc[i][jj] = __fmaf_rn(-av[i], bv[jj], acc[i][jj]);
+        }
+        __syncthreads();                             // every thread is done with buffer ch & 1
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i) {
+        const int64_t r = r0 + tr + (i & 3) + (i >> 2) * 64;
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const int64_t r = r0 + tr + i, cc = c0 + tc + jj;
+        for (int jj = 0; jj < 8; ++jj) {
+            const int64_t cc = c0 + tc + (jj & 3) + (jj >> 2) * 64;
             if (r < rows && cc < cols) w[r * cols + cc] = acc[i][jj];
         }
+    }
 }
 
 }  // namespace
 
-size_t gptq_workspace_bytes(int64_t rows) { return (size_t)rows * kB * sizeof(float); }
+// Workspace: the block's scaled errors, transposed ([128][ldE] with ldE the
+// row count rounded up to a multiple of 4, so every 16-byte copy is aligned).
+static int64_t gptq_ld(int64_t rows) { return (rows + 3) / 4 * 4; }
+
+size_t gptq_workspace_bytes(int64_t rows) { return (size_t)gptq_ld(rows) * kB * sizeof(float); }
 
 cudaError_t launch_nvfp4_gptq(float* w, int64_t rows, int64_t cols, const float* U, const float* d_amax,
                               uint8_t* codes, uint8_t* scales, float* d_S, float* deq, float* E, int32_t* d_status,
                               cudaStream_t s)
 {
-    const size_t smem_a_max = (size_t)(kRowsA * (kB + 1) + kB * kB) * sizeof(float);
-    const size_t smem_b_max = (size_t)(2 * kB * kTile) * sizeof(float);
+    const size_t smem_a_max = (size_t)kB * kB * sizeof(float);
+    const size_t smem_b = (size_t)4 * kBK * kTB * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(gptq_block_kernel),
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a_max);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(reinterpret_cast<const void*>(gptq_update_kernel),
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b_max);
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b);
     if (e != cudaSuccess) return e;
-    const unsigned grid_a = (unsigned)((rows + kRowsA - 1) / kRowsA);
+    const int64_t ldE = gptq_ld(rows);
+    const unsigned grid_a = (unsigned)((rows + (kThreadsA / kLanes) - 1) / (kThreadsA / kLanes));
     for (int64_t j0 = 0; j0 < cols; j0 += kB) {
         const int bw = (int)(cols - j0 < kB ? cols - j0 : kB);
-        const size_t smem_a = (size_t)(kRowsA * (bw + 1) + bw * bw) * sizeof(float);
-        gptq_block_kernel<<<grid_a, kRowsA, smem_a, s>>>(w, rows, cols, j0, bw, U, d_amax, codes, scales, d_S, deq, E,
-                                                         d_status, -0.0f);
+        const size_t smem_a = (size_t)bw * bw * sizeof(float);
+        gptq_block_kernel<<<grid_a, kThreadsA, smem_a, s>>>(w, rows, cols, j0, bw, U, d_amax, codes, scales, d_S,
+                                                            deq, E, ldE, d_status, -0.0f);
         const int64_t rem = cols - j0 - bw;
         if (rem > 0) {
-            const dim3 grid_b((unsigned)((rows + kTile - 1) / kTile), (unsigned)((rem + kTile - 1) / kTile));
-            const size_t smem_b = (size_t)(2 * bw * kTile) * sizeof(float);
-            gptq_update_kernel<<<grid_b, 256, smem_b, s>>>(w, rows, cols, j0, bw, U, E);
+            const dim3 grid_b((unsigned)((rows + kTB - 1) / kTB), (unsigned)((rem + kTB - 1) / kTB));
+            gptq_update_kernel<<<grid_b, 256, smem_b, s>>>(w, rows, cols, j0, bw, U, E, ldE);
         }
     }
     return cudaGetLastError();
