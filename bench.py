@@ -371,9 +371,9 @@ def run_reference(args):
 # (profiles/nvfp4_sweep_mse_16384x8192.md).  Traffic grows in proportion to the
 # elements, so a launch of n elements moves about n times this.  Once the sources
 # differ the figure no longer describes the kernel and none is reported.
-NVFP4_TRAFFIC = {"bytes_per_element": 556360704 / (16384 * 8192),
+NVFP4_TRAFFIC = {"bytes_per_element": (268480768 + 286225664) / (16384 * 8192),
                  "sources": ("nvfp4.cu", "nvfp4_block.cuh", "screen.cuh", "device.cuh"),
-                 "sha256": "6bca92bddfc55825b97e6db03fd9f5ecf560acb991e9d7009fe272f1d38c7bb8"}
+                 "sha256": "eeaccfe992e1af1b0984c8a9ffe3cbcc1d13d088c6b8c2383109abd62a785fc2"}
 
 
 def measured_traffic_per_launch(elements_per_launch):
