@@ -49,7 +49,8 @@
  *           caller zeroes it before the calls and reads it after a
  *           synchronize.  When a flag is set the outputs are unspecified.
  * Numerics. All arithmetic is IEEE binary32 with round-to-nearest-even, no
- *           fused multiply-add and no flush-to-zero.  Each block's loss is
+ *           fused multiply-add (except the error updates that
+ *           fp4q_nvfp4_gptq defines as fused) and no flush-to-zero.  Each block's loss is
  *           accumulated sequentially over its elements in column order:
  *             r = x*inv; q = E2M1(r); y = q*d; e = x - y;
  *             MSE: L = L + e*e        WMSE: L = L + w[col]*(e*e)
