@@ -30,7 +30,7 @@ __all__ = [
     "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes", "nvfp4_quantize_dynamic",
     "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout", "mma_scales",
     "fp4q_focus_quant", "fp4q_mxfp4_unrotate", "focus_quantize", "mxfp4_unrotate", "FocusResult",
-    "fp4q_nvfp4_gptq", "fp4q_gptq_workspace_bytes", "nvfp4_gptq",
+    "fp4q_nvfp4_gptq", "fp4q_gptq_workspace_bytes", "nvfp4_gptq", "fp4q_probe_wait",
     "quantize_batch",
     "NVFP4Result", "MXFP4Result", "nvfp4_quantize", "mxfp4_quantize", "quantize_dual", "dequantize",
     "FLAG_NONFINITE", "FLAG_RANGE", "FLAG_TIMEOUT",
@@ -52,7 +52,7 @@ EXPORTS = ("fp4q_version", "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_g
            "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_quantize_batch_static", "fp4q_dequant",
            "fp4q_probe_e2m1", "fp4q_probe_e4m3", "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes",
            "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout", "fp4q_focus_quant", "fp4q_mxfp4_unrotate",
-           "fp4q_nvfp4_gptq", "fp4q_gptq_workspace_bytes")
+           "fp4q_nvfp4_gptq", "fp4q_gptq_workspace_bytes", "fp4q_probe_wait")
 
 
 class BatchTensor(ctypes.Structure):
@@ -107,6 +107,7 @@ def load():
         "fp4q_dequant": [I, P, P, P, I64, I64, P, I, P],
         "fp4q_probe_e2m1": [P, P, I64, P],
         "fp4q_probe_e4m3": [P, P, I64, P],
+        "fp4q_probe_wait": [P, ctypes.c_uint32, ctypes.c_uint32, P, P],
     }
     sigs["fp4q_quantize_batch"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, ctypes.c_size_t, P, P]
     sigs["fp4q_quantize_batch_static"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, P]
@@ -474,6 +475,14 @@ def fp4q_probe_e2m1(r: torch.Tensor, out: torch.Tensor, stream=None) -> None:
     _check(load().fp4q_probe_e2m1(_dev(r, "r", torch.float32, device=dev),
                                   _dev(out, "out", torch.uint8, r.numel(), dev), r.numel(),
                                   _stream(stream)), "fp4q_probe_e2m1")
+
+
+def fp4q_probe_wait(flag: torch.Tensor, target: int, limit: int, d_status: torch.Tensor, stream=None) -> None:
+    """The library's bounded spin-wait on its own (diagnostic): wait for
+    flag >= target at most `limit` polls, FLAG_TIMEOUT in d_status if not."""
+    fp = _dev(flag, "flag", (torch.int32, torch.uint32), 1, flag.device)
+    sp = _dev(d_status, "d_status", torch.int32, 1, flag.device)
+    _check(load().fp4q_probe_wait(fp, int(target), int(limit), sp, _stream(stream)), "fp4q_probe_wait")
 
 
 def fp4q_probe_e4m3(v: torch.Tensor, out: torch.Tensor, stream=None) -> None:

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp4q.so")
 SOURCES = ["api.cu", "absmax.cu", "nvfp4.cu", "mxfp4.cu", "dequant.cu", "batch.cu", "dynamic.cu", "layout.cu", "focus.cu", "gptq.cu"]
-HEADERS = ["device.cuh", "launch.h", "screen.cuh", "nvfp4_block.cuh", "mxfp4_block.cuh", "batch.h"]
+HEADERS = ["device.cuh", "launch.h", "screen.cuh", "nvfp4_block.cuh", "mxfp4_block.cuh", "batch.h", "wait.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -459,6 +459,16 @@ fp4q_status fp4q_probe_e2m1(const float* r, uint8_t* out, int64_t n, fp4q_stream
     return after_launch();
 }
 
+fp4q_status fp4q_probe_wait(const uint32_t* flag, uint32_t target, uint32_t limit, int32_t* d_status,
+                            fp4q_stream_t stream)
+{
+    if (!flag || !d_status) return FP4Q_ERR_NULL;
+    if (!aligned(flag, 4) || !aligned(d_status, 4)) return FP4Q_ERR_ALIGN;
+    if (limit > (1u << 24)) return FP4Q_ERR_ARG;
+    fp4q::launch_probe_wait(flag, target, limit, d_status, reinterpret_cast<cudaStream_t>(stream));
+    return after_launch();
+}
+
 fp4q_status fp4q_probe_e4m3(const float* v, uint8_t* out, int64_t n, fp4q_stream_t stream)
 {
     if (n < 0) return FP4Q_ERR_SHAPE;

@@ -25,6 +25,7 @@
 #include "launch.h"
 #include "mxfp4_block.cuh"
 #include "nvfp4_block.cuh"
+#include "wait.cuh"
 
 namespace fp4q {
 
@@ -33,7 +34,6 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kMxBlocksPerThread = 2;   // 512 MXFP4 blocks = 16384 elements per tile
 constexpr int kNvBlocksPerThread = 4;   // 1024 NVFP4 blocks = 16384 elements per tile
-constexpr unsigned kWaitLimit = 1u << 24;
 
 __device__ __forceinline__ unsigned ld_volatile(const unsigned* p)
 {
@@ -111,14 +111,10 @@ batch_kernel(const __grid_constant__ BatchParams P, unsigned* __restrict__ ws, i
         } else {
             // ---------------- NVFP4 tile of weight t: wait for its max
             if (threadIdx.x == 0) {
-                unsigned it = 0, skip = 0;
-                while (ld_volatile(done + t) < (unsigned)P.mx_tiles[t]) {
-                    if (++it > kWaitLimit) {
-                        atomicOr(d_status, kFlagTimeout);
-                        skip = 1;
-                        break;
-                    }
-                    __nanosleep(128);
+                unsigned skip = 0;
+                if (!wait_geq(done + t, (unsigned)P.mx_tiles[t], kWaitLimit)) {
+                    atomicOr(d_status, kFlagTimeout);
+                    skip = 1;
                 }
                 __threadfence();
                 s_gmax = ld_volatile(gmax + t);

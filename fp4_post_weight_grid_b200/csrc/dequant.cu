@@ -10,6 +10,7 @@
 
 #include "device.cuh"
 #include "launch.h"
+#include "wait.cuh"
 
 namespace fp4q {
 
@@ -62,6 +63,14 @@ dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
     }
 }
 
+// The library's bounded spin-wait on its own: one thread waits for *flag >=
+// target and raises FP4Q_FLAG_TIMEOUT if that does not happen within `limit`
+// polls, so that tests can watch a wait run out without any fault.
+__global__ void probe_wait_kernel(const unsigned* flag, unsigned target, unsigned limit, int32_t* d_status)
+{
+    if (!wait_geq(flag, target, limit)) atomicOr(d_status, kFlagTimeout);
+}
+
 __global__ void probe_e2m1_kernel(const float* __restrict__ r, uint8_t* __restrict__ out, int64_t n)
 {
     const int64_t npair = (n + 1) / 2;
@@ -112,6 +121,11 @@ void launch_dequant(bool mx, const uint8_t* codes, const uint8_t* scales, const 
             dequant_kernel<float, false><<<g, kThreads, 0, s>>>(codes, scales, d_S, nb,
                                                                 static_cast<float*>(out));
     }
+}
+
+void launch_probe_wait(const unsigned* flag, unsigned target, unsigned limit, int32_t* d_status, cudaStream_t s)
+{
+    probe_wait_kernel<<<1, 1, 0, s>>>(flag, target, limit, d_status);
 }
 
 void launch_probe_e2m1(const float* r, uint8_t* out, int64_t n, cudaStream_t s)

@@ -34,6 +34,7 @@
 #include "device.cuh"
 #include "launch.h"
 #include "nvfp4_block.cuh"
+#include "wait.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -42,7 +43,6 @@ namespace fp4q {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr unsigned kWaitLimit = 1u << 24;
 
 __device__ __forceinline__ unsigned ld_volatile(const unsigned* p)
 {
@@ -88,14 +88,10 @@ nvfp4_dynamic_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_pe
             if (m != 0u) atomicMax(ws, m);
             __threadfence();
             atomicAdd(ws + 1, 1u);
-            unsigned it = 0, skip = 0;
-            while (ld_volatile(ws + 1) < gridDim.x) {
-                if (++it > kWaitLimit) {
-                    atomicOr(d_status, kFlagTimeout);
-                    skip = 1;
-                    break;
-                }
-                __nanosleep(128);
+            unsigned skip = 0;
+            if (!wait_geq(ws + 1, gridDim.x, kWaitLimit)) {
+                atomicOr(d_status, kFlagTimeout);
+                skip = 1;
             }
             __threadfence();
             s_gmax = ld_volatile(ws);

@@ -493,6 +493,19 @@ fp4q_status fp4q_dequant(fp4q_format format, const uint8_t* codes, const uint8_t
 fp4q_status fp4q_probe_e2m1(const float* r, uint8_t* out, int64_t n, fp4q_stream_t stream);
 fp4q_status fp4q_probe_e4m3(const float* v, uint8_t* out, int64_t n, fp4q_stream_t stream);
 
+/*
+ * fp4q_probe_wait -- diagnostic with no counterpart in the papers: the
+ * library's bounded spin-wait (the one the batch kernel and the one-launch
+ * sweep use to wait for other thread blocks) run by one thread on its own.
+ * It polls *flag until it is at least `target`, at most `limit` times about
+ * 128 ns apart, and raises FP4Q_FLAG_TIMEOUT in *d_status if it gave up; so a
+ * test can watch a wait run out and the context stay usable.
+ *   flag      device uint32 (4-byte aligned), read only.
+ *   limit     at most 2^24 (the library's own limit), else FP4Q_ERR_ARG.
+ */
+fp4q_status fp4q_probe_wait(const uint32_t* flag, uint32_t target, uint32_t limit, int32_t* d_status,
+                            fp4q_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
