@@ -551,6 +551,129 @@ def run_act_latency(args):
     return 0
 
 
+# --------------------------------------------------------------------------- per-workload records
+
+def run_configs(args):
+    """One JSON record per small workload (not the benchmark line): the
+    outlier matrix (128 x 256 fp32, NVFP4-MSE), the q_proj-shaped 4096 x 4096
+    (NVFP4-MSE), the WMSE 11008 x 4096 with its importance vector and the
+    rotated MXFP4 28672 x 8192 (the whole-model pass is the benchmark line).
+    Per record: the ABI sequence (global absmax + sweep, or the rotated MXFP4
+    pass) timed with CUDA events, median of `--steps` launches after
+    `--warmup`, a 512 MB buffer rewritten between launches so that no launch
+    starts with its input in L2; algorithmic bytes and their fraction of the
+    measured HBM peak; parity with the oracle on sampled rows (all rows of
+    the outlier matrix), element by element; the aggregate reconstruction MSE
+    of those rows on both sides (fp64); the oracle's time on those rows."""
+    import fp4_post_weight_grid_b200 as fq
+    from fp4_post_weight_grid_b200 import build as fbuild
+    import oracle
+    import synth
+    fbuild.build()
+    oracle.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hbm_peak, peak_kind, _ = load_peaks()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    reps = max(args.steps, 5)
+
+    def timed(fn):
+        ts = []
+        for i in range(max(args.warmup, 3) + reps):
+            flush.fill_(i & 0xFF)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            if i >= max(args.warmup, 3):
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    def bits(t):
+        t = t.detach().cpu()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+    workloads = [
+        ("outliers 128x256 fp32, NVFP4-MSE", lambda: synth.small_outliers(), None, None, "nv"),
+        ("q_proj 4096x4096 bf16, NVFP4-MSE", lambda: synth.q_proj(4096, 4096, seed=2, device=dev), None, None,
+         "nv"),
+        ("WMSE 11008x4096 bf16, NVFP4-WMSE",
+         lambda: synth.t_weight(11008, 4096, nu=4, scale=0.02, seed=3, device=dev),
+         lambda: synth.importance_diag_xtx(cols=4096, tokens=2048, seed=3), None, "nv"),
+        ("MXFP4+Hadamard 28672x8192 bf16", lambda: synth.t_weight(28672, 8192, nu=3, scale=0.015, seed=4,
+                                                                 device=dev),
+         None, lambda: synth.sign_masks(8192, seed=4), "mx"),
+    ]
+    for name, make_w, make_imp, make_masks, kind in workloads:
+        w = make_w().to(dev)
+        rows, cols = w.shape
+        n = rows * cols
+        isz = w.element_size()
+        imp_np = make_imp().numpy() if make_imp else None
+        imp = torch.from_numpy(imp_np).to(dev) if make_imp else None
+        masks_np = make_masks() if make_masks else None
+        masks = torch.from_numpy(masks_np.view(np.int32)).to(dev) if make_masks else None
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+        deq = torch.empty_like(w)
+        if kind == "nv":
+            amax = torch.empty(1, device=dev)
+            S = torch.empty(1, device=dev)
+            scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+
+            def fn():
+                fq.fp4q_global_absmax(w, amax, stream)
+                if imp is None:
+                    fq.fp4q_nvfp4_sweepmse(w, amax, codes, scales, S, deq, None, st, stream)
+                else:
+                    fq.fp4q_nvfp4_sweepwmse(w, amax, imp, codes, scales, S, deq, None, st, stream)
+            nbytes = n * (isz + isz + 0.5 + 1.0 / 16 + isz)
+        else:
+            scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
+
+            def fn():
+                fq.fp4q_mxfp4_quant_hadamard(w, masks, codes, scales, deq, None, st, stream)
+            nbytes = n * (isz + 0.5 + 1.0 / 32 + isz)
+        ms = timed(fn)
+        # parity on sampled rows
+        idx = np.arange(rows) if rows <= 128 else np.array([0, 1, rows // 2, rows - 1])
+        x_all = w.float().cpu().numpy()
+        x = np.ascontiguousarray(x_all[idx])
+        t0 = time.perf_counter()
+        if kind == "nv":
+            S_o = oracle.global_scale(oracle.global_absmax(x_all))
+            window = oracle.NVFP4_WMSE_WINDOW if imp_np is not None else oracle.NVFP4_MSE_WINDOW
+            o = oracle.nvfp4_quant(x, S=S_o, importance=imp_np, window=window)
+        else:
+            o = oracle.mxfp4_quant(x, sign_masks=masks_np)
+        t_orc = time.perf_counter() - t0
+        deq_o = oracle.bf16_round(o["y"]) if w.dtype == torch.bfloat16 else o["y"]
+        dg = bits(deq)[idx]
+        same = (np.array_equal(bits(codes)[idx], o["codes"]) and np.array_equal(bits(scales)[idx], o["scales"])
+                and np.array_equal(dg.view(np.uint32) if dg.dtype == np.float32 else dg,
+                                   deq_o.view(np.uint32) if deq_o.dtype == np.float32 else deq_o))
+        ref = o["rotated"] if kind == "mx" else x
+        y_gpu = deq.float().cpu().numpy()[idx].astype(np.float64)
+        y_orc = (deq_o.astype(np.uint32) << 16).view(np.float32).astype(np.float64) \
+            if w.dtype == torch.bfloat16 else deq_o.astype(np.float64)
+        mse_gpu = float(np.mean((ref.astype(np.float64) - y_gpu) ** 2))
+        mse_orc = float(np.mean((ref.astype(np.float64) - y_orc) ** 2))
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        print(json.dumps({"workload": name, "shape": [rows, cols], "ms": ms, "input_gbs": n * isz / (ms * 1e-3) / 1e9,
+                          "elements_per_s": n / (ms * 1e-3), "algorithmic_bytes": nbytes, "algorithmic_gbs": gbs,
+                          "hbm_frac": gbs / hbm_peak, "peak_kind": peak_kind, "status": int(st.item()),
+                          "parity_rows": int(idx.size), "parity_bit_exact": bool(same),
+                          "mse_gpu": mse_gpu, "mse_oracle": mse_orc,
+                          "mse_rel_diff": abs(mse_gpu - mse_orc) / max(mse_orc, 1e-300),
+                          "oracle_s_on_rows": t_orc, "oracle_cores": oracle.max_threads()}), flush=True)
+        del w, deq, codes
+        torch.cuda.empty_cache()
+    return 0
+
+
 # --------------------------------------------------------------------------- GPTQ
 
 def run_gptq(args):
@@ -623,6 +746,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", action="store_true",
+                    help="one JSON record per small workload: time, bytes, roofline, parity, MSE, oracle time")
     ap.add_argument("--gptq", action="store_true",
                     help="time the ScaleSweep inside GPTQ on one weight (default 11008x4096)")
     ap.add_argument("--act-latency", action="store_true",
@@ -646,6 +771,8 @@ def main():
         return run_single(args)
     if args.act_latency:
         return run_act_latency(args)
+    if args.configs:
+        return run_configs(args)
     if args.gptq:
         if args.shape == "16384x8192":
             args.shape = "11008x4096"
