@@ -17,7 +17,10 @@
 // the same time, and the whole list costs one launch.
 //
 // The per-block arithmetic is exactly that of the single-weight kernels
-// (nvfp4_block.cuh, mxfp4_block.cuh), so the results are bit-identical.
+// (nvfp4_block.cuh, mxfp4_block.cuh), so the results are bit-identical.  The
+// MXFP4 tiles use the neighbour-paired form for both plain and rotated
+// blocks: one kernel holds both, and the half-paired form's extra registers
+// would spill here.
 #include <mutex>
 
 #include "batch.h"
@@ -89,10 +92,10 @@ batch_kernel(const __grid_constant__ BatchParams P, unsigned* __restrict__ ws, i
                 float* ls = d.mx_loss ? d.mx_loss + b : nullptr;
                 uint32_t bm;
                 if (d.sign_masks)
-                    bm = mxfp4_block<T, true>(src, __ldg(d.sign_masks + (b % bpr)), d.mx_codes + b * 16,
+                    bm = mxfp4_block_pairs_of_neighbours<T, true>(src, __ldg(d.sign_masks + (b % bpr)), d.mx_codes + b * 16,
                                               d.mx_scales + b, dq, ls, d_status, z2, neg_zero);
                 else
-                    bm = mxfp4_block<T, false>(src, 0u, d.mx_codes + b * 16, d.mx_scales + b, dq, ls,
+                    bm = mxfp4_block_pairs_of_neighbours<T, false>(src, 0u, d.mx_codes + b * 16, d.mx_scales + b, dq, ls,
                                                d_status, z2, neg_zero);
                 m = max(m, bm);
             }

@@ -28,13 +28,9 @@ namespace fp4q {
 
 constexpr float kInvSqrt32 = 0x1.6a09e6p-3f;   // RN(1/sqrt(32))
 
-// Quantize one 32-element block; returns max|w| (as binary32 bits) of the
-// unrotated block, for a fused global max.
-//   src      the block's 32 input elements; sign_mask: its sign mask (HAD only)
-//   codes16  16 bytes of packed nibbles; scale: the E8M0 byte
-//   deq32    32 reconstructed elements or nullptr; loss: the block's loss or nullptr
+// Neighbour-paired form (elements 2j, 2j+1 in a register pair).
 template <typename T, bool HAD>
-__device__ __forceinline__ uint32_t mxfp4_block(const T* __restrict__ src, uint32_t sign_mask,
+__device__ __forceinline__ uint32_t mxfp4_block_pairs_of_neighbours(const T* __restrict__ src, uint32_t sign_mask,
                                                 uint8_t* __restrict__ codes16, uint8_t* __restrict__ scale,
                                                 T* __restrict__ deq32, float* __restrict__ loss,
                                                 int32_t* __restrict__ d_status, uint64_t z2, float neg_zero)
@@ -176,6 +172,225 @@ __device__ __forceinline__ uint32_t mxfp4_block(const T* __restrict__ src, uint3
     if (loss) *loss = L;
     return wmax;
 
+}
+
+// Half-paired form (elements j, j+16 in a register pair), for the rotation.
+template <typename T, bool HAD>
+__device__ __forceinline__ uint32_t mxfp4_block_pairs_of_halves(const T* __restrict__ src, uint32_t sign_mask,
+                                                uint8_t* __restrict__ codes16, uint8_t* __restrict__ scale,
+                                                T* __restrict__ deq32, float* __restrict__ loss,
+                                                int32_t* __restrict__ d_status, uint64_t z2, float neg_zero)
+{
+    // The block lives in 16 register pairs P[j].  With the rotation, P[j]
+    // holds elements j and j+16: the butterfly stages h = 1, 2, 4, 8 act on
+    // both alike and run as packed adds, stage h = 16 combines the two halves
+    // of each pair; every element sees the operations of the stage-by-stage
+    // definition in its order.  (Without the rotation P[j] would hold the
+    // neighbours 2j, 2j+1.)  The search and the emit work on whatever pairing
+    // P has; E(j, h) is the element held in half h of P[j].
+#define FP4Q_E(j, h) (HAD ? (j) + 16 * (h) : 2 * (j) + (h))
+    float x[32];
+    uint32_t wmax;         // max |w| bits of the unrotated block
+    load_block_amax<32>(src, x, wmax);
+    uint32_t abits = wmax; // max |y| bits of the block that is quantized
+    uint64_t P[16];
+    if (HAD) {
+        const uint32_t m = sign_mask;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            x[j] = __uint_as_float(__float_as_uint(x[j]) ^ (((m >> j) & 1u) << 31));
+#pragma unroll
+        for (int j = 0; j < 16; ++j) P[j] = pk(x[j], x[j + 16]);
+#pragma unroll
+        for (int h = 1; h < 16; h *= 2) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if (i & h) continue;
+                const uint64_t a = P[i], c = P[i + h];
+                P[i] = add2(a, c);
+                P[i + h] = sub2(a, c);
+            }
+        }
+        const uint64_t c2 = pk(kInvSqrt32, kInvSqrt32);
+        abits = 0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float a, c;
+            upk(P[j], a, c);
+            P[j] = mul2(pk(__fadd_rn(a, c), __fsub_rn(a, c)), c2);
+            upk(P[j], a, c);
+            abits = max(abits, max(__float_as_uint(a) & 0x7FFFFFFFu, __float_as_uint(c) & 0x7FFFFFFFu));
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) P[j] = pk(x[2 * j], x[2 * j + 1]);
+    }
+    // From here on the search works on the signed values: E2M1 rounding and
+    // every loss term are symmetric in the sign.
+    if (abits >= 0x7F800000u) atomicOr(d_status, kFlagNonfinite);
+    int e0 = -127;
+    if (abits >= 0x00800000u) {
+        const int a = (int)(abits >> 23) - 127;                 // floor(log2 amax)
+        e0 = a - 2 + ((abits & 0x7FFFFFu) > 0x400000u ? 1 : 0);  // 6*2^(a-2) = 1.5*2^a
+        e0 = min(max(e0, -127), 127);
+    }
+    // candidate k = 0, 1, 2 is the exponent e0 - 1 + k, clamped to [-127, 127]
+#define FP4Q_EK(k) min(max(e0 - 1 + (k), -127), 127)
+
+    // 1. screen the three exponents in units of 2^e0 (S = 2^e0, v = 2^(e-e0))
+    const float inv0 = exp2i(-e0);
+    const float as = __uint_as_float(abits) * inv0;      // sum y^2 / S^2 <= 32 amax^2 / S^2
+    const float alpha2 = (32.0f * as * as) * (1.0f + 0x1p-16f);
+    const float tS = 0x1p-70f * inv0;
+    const float tau = tS * tS + 0x1p-120f;
+    float lam[3];
+    {   // the three exponents, one register pair at a time
+        uint64_t inv2[3], L2[3];
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const float ik = exp2i(-FP4Q_EK(k));
+            inv2[k] = pk(ik, ik);
+            L2[k] = pk(0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+#pragma unroll
+            for (int k = 0; k < 3; ++k) {
+                float ra, rb;
+                upk(mul2(P[j], inv2[k]), ra, rb);
+                const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
+                L2[k] = fma2(et, et, L2[k]);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            float lo, hi;
+            upk(L2[k], lo, hi);
+            lam[k] = (lo + hi) * exp2i(2 * (FP4Q_EK(k) - e0));
+        }
+    }
+    const float M = fminf(fminf(lam[0], lam[1]), lam[2]);
+    const float thr = survivor_threshold(M, alpha2, tau);
+    uint32_t mask = (lam[0] <= thr ? 1u : 0u) | (lam[1] <= thr ? 2u : 0u) | (lam[2] <= thr ? 4u : 0u);
+    if (mask == 0) mask = 7u;                  // unreachable for finite inputs; evaluate all
+
+    // 2. verify: exact loss of the survivors (summed in element order), first minimum wins
+    int be;
+    if ((mask & (mask - 1)) == 0) {
+        be = FP4Q_EK(__ffs(mask) - 1);
+    } else {
+        float best = 0.0f;
+        bool first = true;
+        be = FP4Q_EK(0);
+        while (mask) {
+            const int k = __ffs(mask) - 1;
+            mask &= mask - 1;
+            const int e = FP4Q_EK(k);
+            const uint64_t d2 = pk(exp2i(e), exp2i(e)), inv2 = pk(exp2i(-e), exp2i(-e));
+            float s[32];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                float r0, r1;
+                upk(mul2(P[j], inv2), r0, r1);
+                const uint64_t q2 = h2_to_f2(e2m1x2_round_h(r0, r1), neg_zero);
+                const uint64_t e2 = sub2(P[j], mul2_nofuse(q2, d2, z2));
+                upk(mul2_nofuse(e2, e2, z2), s[FP4Q_E(j, 0)], s[FP4Q_E(j, 1)]);
+            }
+            float L = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) L = __fadd_rn(L, s[i]);
+            if (first || L < best) { best = L; be = e; }
+            first = false;
+        }
+    }
+
+    // 3. emit the winner: codes, reconstruction q*d and, when requested, its
+    //    exact loss in element order
+    const float d = exp2i(be), inv = exp2i(-be);
+    const uint64_t d2 = pk(d, d), inv2 = pk(inv, inv);
+    uint32_t word[4];
+    float L = 0.0f;
+    // one 8-element chunk: its 8 quotients in element order -> word[c] and deq
+    auto emit_chunk = [&](int c, const float (&rc)[8]) {
+        float y[8];
+        uint32_t q2[4];
+        word[c] = e2m1x8_encode(rc, q2);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) upk(mul2_nofuse(f16x2_to_f2(q2[j]), d2, z2), y[2 * j], y[2 * j + 1]);
+        if (deq32) store_block<8>(deq32 + 8 * c, y);
+    };
+    if (HAD) {
+        // pairs 8g..8g+7 hold elements 8g..8g+7 (low halves, chunk g) and
+        // 16+8g..16+8g+7 (high halves, chunk 2+g)
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            float rl[8], rh[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) upk(mul2(P[8 * g + m], inv2), rl[m], rh[m]);
+            emit_chunk(g, rl);
+            emit_chunk(2 + g, rh);
+        }
+        if (loss) {     // the winner is known; its exact loss is only an output
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                float lo, hi;
+                upk(P[i & 15], lo, hi);
+                const float xi = i < 16 ? lo : hi;
+                const uint32_t code = e2m1x2(__fmul_rn(xi, inv), 0.0f) & 0xFu;
+                float q, unused;
+                f16x2_to_f32(e2m1x2_to_f16x2(code), q, unused);
+                const float e = __fsub_rn(xi, __fmul_rn(q, d));
+                L = __fadd_rn(L, __fmul_rn(e, e));
+            }
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float rc[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) upk(mul2(P[4 * c + j], inv2), rc[2 * j], rc[2 * j + 1]);
+            emit_chunk(c, rc);
+        }
+        if (loss) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                float r0, r1;
+                upk(mul2(P[j], inv2), r0, r1);
+                const uint64_t y2 = mul2_nofuse(e2m1x2_decode(e2m1x2(r0, r1)), d2, z2);
+                const uint64_t e2 = sub2(P[j], y2);
+                float s0, s1;
+                upk(mul2_nofuse(e2, e2, z2), s0, s1);
+                L = __fadd_rn(__fadd_rn(L, s0), s1);
+            }
+        }
+    }
+#undef FP4Q_E
+#undef FP4Q_EK
+    st_stream(codes16, make_uint4(word[0], word[1], word[2], word[3]));
+    *scale = (uint8_t)(be + 127);
+    if (loss) *loss = L;
+    return wmax;
+
+}
+
+// Quantize one 32-element block; returns max|w| (as binary32 bits) of the
+// unrotated block, for a fused global max.
+//   src      the block's 32 input elements; sign_mask: its sign mask (HAD only)
+//   codes16  16 bytes of packed nibbles; scale: the E8M0 byte
+//   deq32    32 reconstructed elements or nullptr; loss: the block's loss or nullptr
+// Both forms compute the same bytes; the rotated one keeps elements j and j+16
+// in one register pair so that four of the five butterfly stages run packed.
+template <typename T, bool HAD>
+__device__ __forceinline__ uint32_t mxfp4_block(const T* __restrict__ src, uint32_t sign_mask,
+                                                uint8_t* __restrict__ codes16, uint8_t* __restrict__ scale,
+                                                T* __restrict__ deq32, float* __restrict__ loss,
+                                                int32_t* __restrict__ d_status, uint64_t z2, float neg_zero)
+{
+    if constexpr (HAD)
+        return mxfp4_block_pairs_of_halves<T, true>(src, sign_mask, codes16, scale, deq32, loss, d_status, z2, neg_zero);
+    else
+        return mxfp4_block_pairs_of_neighbours<T, false>(src, sign_mask, codes16, scale, deq32, loss, d_status, z2,
+                                                         neg_zero);
 }
 
 }  // namespace fp4q
