@@ -50,13 +50,18 @@ namespace {
 
 thread_local char g_last_cuda_error[256] = "no error";
 
-fp4q_status after_launch()
+// FP4Q_ERR_CUDA for a failed CUDA call, its message kept for fp4q_last_cuda_error.
+fp4q_status cuda_failure(cudaError_t e)
 {
-    const cudaError_t e = cudaGetLastError();
-    if (e == cudaSuccess) return FP4Q_OK;
     std::strncpy(g_last_cuda_error, cudaGetErrorString(e), sizeof(g_last_cuda_error) - 1);
     g_last_cuda_error[sizeof(g_last_cuda_error) - 1] = '\0';
     return FP4Q_ERR_CUDA;
+}
+
+fp4q_status after_launch()
+{
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? FP4Q_OK : cuda_failure(e);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -290,12 +295,7 @@ fp4q_status fp4q_nvfp4_gptq(float* w, int64_t rows, int64_t cols, const float* U
     const cudaError_t e = fp4q::launch_nvfp4_gptq(w, rows, cols, U, d_amax, codes, scales_e4m3, d_global_scale, deq,
                                                   static_cast<float*>(workspace), d_status,
                                                   reinterpret_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) {
-        std::strncpy(g_last_cuda_error, cudaGetErrorString(e), sizeof(g_last_cuda_error) - 1);
-        g_last_cuda_error[sizeof(g_last_cuda_error) - 1] = '\0';
-        return FP4Q_ERR_CUDA;
-    }
-    return FP4Q_OK;
+    return e == cudaSuccess ? FP4Q_OK : cuda_failure(e);
 }
 
 int64_t fp4q_mma_scale_bytes(int64_t rows, int64_t scale_cols)
@@ -344,10 +344,8 @@ fp4q_status fp4q_nvfp4_sweep_dynamic(const void* x, fp4q_dtype dt, int64_t rows,
                                                      scales_e4m3, d_global_scale, deq, block_loss,
                                                      static_cast<unsigned*>(workspace), d_status, s);
     if (e != cudaSuccess) {
-        (void)cudaGetLastError();
-        std::strncpy(g_last_cuda_error, cudaGetErrorString(e), sizeof(g_last_cuda_error) - 1);
-        g_last_cuda_error[sizeof(g_last_cuda_error) - 1] = '\0';
-        return FP4Q_ERR_CUDA;
+        (void)cudaGetLastError();                    // a refused launch configuration is not sticky
+        return cuda_failure(e);
     }
     return after_launch();
 }
