@@ -607,6 +607,8 @@ def run_configs(args):
                                                                  device=dev),
          None, lambda: synth.sign_masks(8192, seed=4), "mx"),
     ]
+    workloads.append(("FOCUS NVFP4 (sub-blocks of 8) 4096x4096 bf16",
+                      lambda: synth.q_proj(4096, 4096, seed=2, device=dev), None, None, "focus"))
     for name, make_w, make_imp, make_masks, kind in workloads:
         w = make_w().to(dev)
         rows, cols = w.shape
@@ -631,6 +633,16 @@ def run_configs(args):
                 else:
                     fq.fp4q_nvfp4_sweepwmse(w, amax, imp, codes, scales, S, deq, None, st, stream)
             nbytes = n * (isz + isz + 0.5 + 1.0 / 16 + isz)
+        elif kind == "focus":
+            nv0 = fq.nvfp4_quantize(w)                       # the stored scales to relax
+            scales = nv0.scales
+            S = nv0.global_scale
+            gen = torch.Generator(device="cpu").manual_seed(8)
+            coeffs = (0.8 + 0.45 * torch.rand((rows, cols // 8), generator=gen)).to(torch.float16).to(dev)
+
+            def fn():
+                fq.fp4q_focus_quant(fq.NVFP4, w, scales, S, coeffs, 8, codes, deq, None, st, stream)
+            nbytes = n * (isz + 1.0 / 16 + 2.0 / 8 + 0.5 + isz)
         else:
             scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
 
@@ -647,12 +659,15 @@ def run_configs(args):
             S_o = oracle.global_scale(oracle.global_absmax(x_all))
             window = oracle.NVFP4_WMSE_WINDOW if imp_np is not None else oracle.NVFP4_MSE_WINDOW
             o = oracle.nvfp4_quant(x, S=S_o, importance=imp_np, window=window)
+        elif kind == "focus":
+            o = oracle.focus_quant(0, x, bits(scales)[idx], coeffs.cpu().numpy()[idx], 8, S=float(S.item()))
         else:
             o = oracle.mxfp4_quant(x, sign_masks=masks_np)
         t_orc = time.perf_counter() - t0
         deq_o = oracle.bf16_round(o["y"]) if w.dtype == torch.bfloat16 else o["y"]
         dg = bits(deq)[idx]
-        same = (np.array_equal(bits(codes)[idx], o["codes"]) and np.array_equal(bits(scales)[idx], o["scales"])
+        same = (np.array_equal(bits(codes)[idx], o["codes"])
+                and (kind == "focus" or np.array_equal(bits(scales)[idx], o["scales"]))
                 and np.array_equal(dg.view(np.uint32) if dg.dtype == np.float32 else dg,
                                    deq_o.view(np.uint32) if deq_o.dtype == np.float32 else deq_o))
         ref = o["rotated"] if kind == "mx" else x
@@ -729,10 +744,21 @@ def run_gptq(args):
     fmas = rows * cols * (cols - 1) / 2
     clk = load_peaks()[2]
     peak = 148 * SM_FP32_LANES * clk * 1e6 / 1e12
+    # the oracle beside it: parity and time on 4 sampled rows (rows are independent)
+    import oracle
+    oracle.build()
+    idx = np.array([0, 1, rows // 2, rows - 1])
+    t0 = time.perf_counter()
+    o = oracle.nvfp4_gptq(w0.cpu().numpy()[idx], U.cpu().numpy(), S=float(S.item()))
+    t_orc = time.perf_counter() - t0
+    got = codes.cpu().numpy()[idx]
     print(json.dumps({"gptq": [rows, cols], "ms_median": med, "ms_min": min(times),
                       "update_fma": fmas, "tfma_per_s": fmas / (med * 1e-3) / 1e12,
                       "fp32_lane_peak_tfma_per_s": peak, "frac": fmas / (med * 1e-3) / 1e12 / peak,
-                      "status": int(st.item())}), flush=True)
+                      "status": int(st.item()), "parity_rows": 4,
+                      "parity_bit_exact": bool(np.array_equal(got, o["codes"]) and
+                                               np.array_equal(scales.cpu().numpy()[idx], o["scales"])),
+                      "oracle_ms_per_row": t_orc / 4 * 1e3, "oracle_cores": oracle.max_threads()}), flush=True)
     return 0
 
 
