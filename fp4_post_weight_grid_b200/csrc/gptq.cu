@@ -188,14 +188,18 @@ gptq_update_kernel(float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0
     const int tr = (threadIdx.x >> 4) * 4, tc = (threadIdx.x & 15) * 4;
     const int nchunks = (bw + kBK - 1) / kBK;
     gptq_load_chunk(sm, sm + kBK * kTB, Et, ldE, U, rows, cols, j0, bw, 0, r0, c0);
+    // the tile's current values, four columns per 16-byte load (cols is a
+    // multiple of 16, so a group of four is all in or all out)
     float acc[8][8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t r = r0 + tr + (i & 3) + (i >> 2) * 64;
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-            const int64_t cc = c0 + tc + (jj & 3) + (jj >> 2) * 64;
-            acc[i][jj] = (r < rows && cc < cols) ? w[r * cols + cc] : 0.0f;
+        for (int h = 0; h < 2; ++h) {
+            const int64_t cc = c0 + tc + 64 * h;
+            float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (r < rows && cc < cols) v = *reinterpret_cast<const float4*>(w + r * cols + cc);
+            acc[i][4 * h + 0] = v.x; acc[i][4 * h + 1] = v.y; acc[i][4 * h + 2] = v.z; acc[i][4 * h + 3] = v.w;
         }
     }
     for (int ch = 0; ch < nchunks; ++ch) {
@@ -228,9 +232,11 @@ gptq_update_kernel(float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0
     for (int i = 0; i < 8; ++i) {
         const int64_t r = r0 + tr + (i & 3) + (i >> 2) * 64;
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-            const int64_t cc = c0 + tc + (jj & 3) + (jj >> 2) * 64;
-            if (r < rows && cc < cols) w[r * cols + cc] = acc[i][jj];
+        for (int h = 0; h < 2; ++h) {
+            const int64_t cc = c0 + tc + 64 * h;
+            if (r < rows && cc < cols)
+                *reinterpret_cast<float4*>(w + r * cols + cc) =
+                    make_float4(acc[i][4 * h + 0], acc[i][4 * h + 1], acc[i][4 * h + 2], acc[i][4 * h + 3]);
         }
     }
 }
