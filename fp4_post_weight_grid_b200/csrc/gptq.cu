@@ -15,7 +15,7 @@
 // in ascending j, whether they are applied column by column or block by
 // block; so the blocked algorithm below writes exactly the bytes of the plain
 // sequential one.  Per block of 128 columns:
-//   gptq_block_kernel   8 threads per row, each holding one 16-column group
+//   gptq_block_kernel   4 threads per row, each holding two 16-column groups
 //                       of the block in registers, U's diagonal block in
 //                       shared memory: the sweep at every group start, the
 //                       column quantization by the group's owner, the error
@@ -30,6 +30,8 @@
 // its definition is a chain of single-rounding fused multiply-adds in a fixed
 // order, which a tensor-core accumulation (another precision and order) would
 // not reproduce.
+#include <type_traits>
+
 #include "device.cuh"
 #include "launch.h"
 #include "nvfp4_block.cuh"
@@ -39,17 +41,32 @@ namespace fp4q {
 namespace {
 
 constexpr int kB = 128;           // columns per block
-constexpr int kLanes = 8;         // threads per row in the in-block kernel: one 16-column group each
-constexpr int kThreadsA = 256;    // 32 rows per thread block
+constexpr int kLanes = 4;         // threads per row in the in-block kernel: two 16-column groups each
+constexpr int kThreadsA = 256;    // 64 rows per thread block
 constexpr int kTB = 128;          // output tile of the update kernel (rows and columns)
 constexpr int kBK = 32;           // block columns per shared-memory chunk of the update kernel
 
-// In-block GPTQ.  Thread `lane` of a row keeps the row's 16 values of group
-// `lane` of the block in registers.  For every column j of group g, the owner
-// (lane g) quantizes it (after the ScaleSweep of the group at its first
-// column), computes e_j and broadcasts it to the row's other lanes with a
-// warp shuffle; every lane then updates its own later columns with
-// w_c = fma(-e_j, U[j][c], w_c), so each value sees the updates in ascending j.
+// fma(-e, u, x) for the 16 values of one group, u from shared memory
+__device__ __forceinline__ void gptq_update16(float (&x)[16], float e, const float* __restrict__ u)
+{
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        const float4 t = *reinterpret_cast<const float4*>(u + 4 * v);
+        x[4 * v + 0] = __fmaf_rn(-e, t.x, x[4 * v + 0]);
+        x[4 * v + 1] = __fmaf_rn(-e, t.y, x[4 * v + 1]);
+        x[4 * v + 2] = __fmaf_rn(-e, t.z, x[4 * v + 2]);
+        x[4 * v + 3] = __fmaf_rn(-e, t.w, x[4 * v + 3]);
+    }
+}
+
+// In-block GPTQ.  Thread `lane` of a row keeps the row's values of groups
+// 2*lane and 2*lane+1 of the block in registers (x0, x1).  For every column j
+// of group G, the owner (lane G/2) quantizes it (after the ScaleSweep of the
+// group at its first column), computes e_j and broadcasts it to the row's
+// other lanes with a warp shuffle; every lane then updates its own later
+// columns with w_c = fma(-e_j, U[j][c], w_c), so each value sees the updates
+// in ascending j.  Eight rows share a warp, so the owner's serial work runs
+// on eight lanes at once.
 __global__ void __launch_bounds__(kThreadsA)
 gptq_block_kernel(const float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0, int bw,
                   const float* __restrict__ U, const float* __restrict__ d_amax, uint8_t* __restrict__ codes,
@@ -75,73 +92,83 @@ gptq_block_kernel(const float* __restrict__ w, int64_t rows, int64_t cols, int64
     const int64_t row = (int64_t)blockIdx.x * (kThreadsA / kLanes) + threadIdx.x / kLanes;
     const int ngroups = bw / 16;
     const bool active = row < rows;
-    const bool mine = active && lane < ngroups;
-    float x[16];
-    if (mine) {
-        const float4* p = reinterpret_cast<const float4*>(w + row * cols + j0 + 16 * lane);
+    const bool has0 = 2 * lane < ngroups, has1 = 2 * lane + 1 < ngroups;
+    float x0[16], x1[16];
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            const float4 t = p[v];
-            x[4 * v + 0] = t.x; x[4 * v + 1] = t.y; x[4 * v + 2] = t.z; x[4 * v + 3] = t.w;
+    for (int h = 0; h < 2; ++h) {
+        float (&xa)[16] = h == 0 ? x0 : x1;
+        if (active && (h == 0 ? has0 : has1)) {
+            const float4* p4 = reinterpret_cast<const float4*>(w + row * cols + j0 + 32 * lane + 16 * h);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const float4 t = p4[v];
+                xa[4 * v + 0] = t.x; xa[4 * v + 1] = t.y; xa[4 * v + 2] = t.z; xa[4 * v + 3] = t.w;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) xa[k] = 0.0f;
         }
-    } else {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) x[k] = 0.0f;
     }
     const uint64_t z2 = pk(neg_zero, neg_zero);
-#pragma unroll 1
-    for (int g = 0; g < ngroups; ++g) {
+    int p = 0;                                       // the owner lane of the group in flight
+    auto run_group = [&](auto H) {
+        constexpr int h = decltype(H)::value;
+        const int G = 2 * p + h;
+        if (G >= ngroups) return;                    // uniform across the warp
+        float (&xa)[16] = h == 0 ? x0 : x1;
         float d = 1.0f, inv = 1.0f;
-        if (lane == g) {                             // the ScaleSweep of the group's current values
+        if (lane == p) {                             // the ScaleSweep of the group's current values
             float wt[16];
             float amax = 0.0f;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[k]));
+            for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(xa[k]));
             const float as = amax * c.invS;
             const float alpha2 = (16.0f * as * as) * (1.0f + 0x1p-16f);
-            const int bp = nvfp4_select<-3, 11, false>(tb, c, x, amax, wt, alpha2, c.tau0, true, z2, neg_zero);
+            const int bp = nvfp4_select<-3, 11, false>(tb, c, xa, amax, wt, alpha2, c.tau0, true, z2, neg_zero);
             const float4 st = tb.step[bp];
             d = st.x;
             inv = st.y;
-            if (active) scales[row * (cols / 16) + (j0 + 16 * g) / 16] = (uint8_t)bp;
+            if (active) scales[row * (cols / 16) + (j0 + 16 * G) / 16] = (uint8_t)bp;
         }
         uint64_t nib = 0;
+        float y4[4];
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
-            const int j = 16 * g + jj;
+            const int j = 16 * G + jj;
             float e = 0.0f;
-            if (lane == g) {
-                const float wj = x[jj];
+            if (lane == p) {
+                const float wj = xa[jj];
                 const uint32_t code = e2m1x2(__fmul_rn(wj, inv), 0.0f) & 0xFu;
                 float q, unused;
                 f16x2_to_f32(e2m1x2_to_f16x2(code), q, unused);
                 const float y = __fmul_rn(q, d);
                 e = __fdiv_rn(__fsub_rn(wj, y), Us[j * bw + j]);
                 nib |= (uint64_t)code << (4 * jj);
+                y4[jj & 3] = y;
                 if (active) {
                     Et[j * ldE + row] = e;
-                    if (deq) deq[row * cols + j0 + j] = y;
+                    if (deq && (jj & 3) == 3)
+                        *reinterpret_cast<float4*>(deq + row * cols + j0 + j - 3) = make_float4(y4[0], y4[1], y4[2], y4[3]);
                 }
             }
-            e = __shfl_sync(0xFFFFFFFFu, e, src0 + g);
-            const float4* u4 = reinterpret_cast<const float4*>(Us + j * bw + 16 * lane);
-            if (lane > g && lane < ngroups) {
+            e = __shfl_sync(0xFFFFFFFFu, e, src0 + p);
+            const float* uj = Us + j * bw + 32 * lane;
+            if (lane > p) {
+                if (has0) gptq_update16(x0, e, uj);
+                if (has1) gptq_update16(x1, e, uj + 16);
+            } else if (lane == p) {
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const float4 u = u4[v];
-                    x[4 * v + 0] = __fmaf_rn(-e, u.x, x[4 * v + 0]);
-                    x[4 * v + 1] = __fmaf_rn(-e, u.y, x[4 * v + 1]);
-                    x[4 * v + 2] = __fmaf_rn(-e, u.z, x[4 * v + 2]);
-                    x[4 * v + 3] = __fmaf_rn(-e, u.w, x[4 * v + 3]);
-                }
-            } else if (lane == g) {
-                const float* uj = Us + j * bw + 16 * g;
-#pragma unroll
-                for (int k = jj + 1; k < 16; ++k) x[k] = __fmaf_rn(-e, uj[k], x[k]);
+                for (int k = jj + 1; k < 16; ++k) xa[k] = __fmaf_rn(-e, uj[16 * h + k], xa[k]);
+                if (h == 0 && has1) gptq_update16(x1, e, uj + 16);
             }
         }
-        if (lane == g && active)
-            *reinterpret_cast<uint64_t*>(codes + (row * cols + j0 + 16 * g) / 2) = nib;
+        if (lane == p && active)
+            *reinterpret_cast<uint64_t*>(codes + (row * cols + j0 + 16 * G) / 2) = nib;
+    };
+#pragma unroll 1
+    for (p = 0; 2 * p < ngroups; ++p) {
+        run_group(std::integral_constant<int, 0>{});
+        run_group(std::integral_constant<int, 1>{});
     }
 }
 
