@@ -402,6 +402,7 @@ SINGLE_PATHS = {
     "focus-nvfp4": (2.0 + 1.0 / 16 + 2.0 / 8 + 0.5 + 2.0, "focus_kernel NVFP4, sub-blocks of 8"),
     "focus-mxfp4": (2.0 + 1.0 / 32 + 2.0 / 8 + 0.5 + 2.0, "focus_kernel MXFP4, sub-blocks of 8"),
     "unrotate": (4.0, "unrotate_kernel (MXFP4 Hadamard inverse, bf16 in and out)"),
+    "copy": (4.0, "probe_copy_kernel (the library's 16-byte streaming loads and stores, bf16 in and out)"),
 }
 
 
@@ -456,6 +457,8 @@ def run_single(args):
             fq.fp4q_mxfp4_unrotate(w, masks, deq, stream)
         elif args.single == "mma-layout":
             fq.fp4q_scales_to_mma_layout(sc16, tiled, stream)
+        elif args.single == "copy":
+            fq.fp4q_probe_copy(w, deq, stream)
         elif args.single == "dequant-nvfp4":
             fq.fp4q_dequant(fq.NVFP4, codes, sc16, S, rows, cols, deq, stream)
 

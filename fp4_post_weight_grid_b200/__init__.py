@@ -30,7 +30,7 @@ __all__ = [
     "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes", "nvfp4_quantize_dynamic",
     "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout", "mma_scales",
     "fp4q_focus_quant", "fp4q_mxfp4_unrotate", "focus_quantize", "mxfp4_unrotate", "FocusResult",
-    "fp4q_nvfp4_gptq", "fp4q_gptq_workspace_bytes", "nvfp4_gptq", "fp4q_probe_wait",
+    "fp4q_nvfp4_gptq", "fp4q_gptq_workspace_bytes", "nvfp4_gptq", "fp4q_probe_wait", "fp4q_probe_copy",
     "quantize_batch",
     "NVFP4Result", "MXFP4Result", "nvfp4_quantize", "mxfp4_quantize", "quantize_dual", "dequantize",
     "FLAG_NONFINITE", "FLAG_RANGE", "FLAG_TIMEOUT",
@@ -52,7 +52,8 @@ EXPORTS = ("fp4q_version", "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_g
            "fp4q_quantize_batch", "fp4q_batch_workspace_bytes", "fp4q_quantize_batch_static", "fp4q_dequant",
            "fp4q_probe_e2m1", "fp4q_probe_e4m3", "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes",
            "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout", "fp4q_focus_quant", "fp4q_mxfp4_unrotate",
-           "fp4q_nvfp4_gptq", "fp4q_gptq_workspace_bytes", "fp4q_probe_wait")
+           "fp4q_nvfp4_gptq", "fp4q_gptq_workspace_bytes", "fp4q_probe_wait",
+           "fp4q_probe_copy")
 
 
 class BatchTensor(ctypes.Structure):
@@ -108,6 +109,7 @@ def load():
         "fp4q_probe_e2m1": [P, P, I64, P],
         "fp4q_probe_e4m3": [P, P, I64, P],
         "fp4q_probe_wait": [P, ctypes.c_uint32, ctypes.c_uint32, P, P],
+        "fp4q_probe_copy": [P, P, I64, P],
     }
     sigs["fp4q_quantize_batch"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, ctypes.c_size_t, P, P]
     sigs["fp4q_quantize_batch_static"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, P]
@@ -475,6 +477,16 @@ def fp4q_probe_e2m1(r: torch.Tensor, out: torch.Tensor, stream=None) -> None:
     _check(load().fp4q_probe_e2m1(_dev(r, "r", torch.float32, device=dev),
                                   _dev(out, "out", torch.uint8, r.numel(), dev), r.numel(),
                                   _stream(stream)), "fp4q_probe_e2m1")
+
+
+def fp4q_probe_copy(src: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
+    """Plain streaming copy of src's bytes into dst (diagnostic: the copy
+    bandwidth of the library's own loads and stores)."""
+    nbytes = src.numel() * src.element_size()
+    if dst.numel() * dst.element_size() < nbytes:
+        raise ValueError("dst is smaller than src")
+    _check(load().fp4q_probe_copy(_dev(src, "src", device=src.device), _dev(dst, "dst", device=src.device),
+                                  nbytes, _stream(stream)), "fp4q_probe_copy")
 
 
 def fp4q_probe_wait(flag: torch.Tensor, target: int, limit: int, d_status: torch.Tensor, stream=None) -> None:

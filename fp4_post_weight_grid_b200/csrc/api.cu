@@ -457,6 +457,16 @@ fp4q_status fp4q_probe_e2m1(const float* r, uint8_t* out, int64_t n, fp4q_stream
     return after_launch();
 }
 
+fp4q_status fp4q_probe_copy(const void* src, void* dst, int64_t bytes, fp4q_stream_t stream)
+{
+    if (bytes < 0 || bytes % 16) return FP4Q_ERR_SHAPE;
+    if (bytes == 0) return FP4Q_OK;
+    if (!src || !dst) return FP4Q_ERR_NULL;
+    if (!aligned(src, 16) || !aligned(dst, 16)) return FP4Q_ERR_ALIGN;
+    fp4q::launch_probe_copy(src, dst, bytes, reinterpret_cast<cudaStream_t>(stream));
+    return after_launch();
+}
+
 fp4q_status fp4q_probe_wait(const uint32_t* flag, uint32_t target, uint32_t limit, int32_t* d_status,
                             fp4q_stream_t stream)
 {

@@ -63,6 +63,25 @@ dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
     }
 }
 
+// A plain streaming copy (16-byte loads and stores, four in flight per
+// thread, grid-stride): the copy bandwidth this library's own loads and
+// stores reach, for the HBM roofline of the benchmark.
+__global__ void __launch_bounds__(kThreads) probe_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                              int64_t n16)
+{
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    for (; i + 3 * stride < n16; i += 4 * stride) {
+        const uint4 a = ld_stream(src + i), b = ld_stream(src + i + stride);
+        const uint4 c = ld_stream(src + i + 2 * stride), d = ld_stream(src + i + 3 * stride);
+        st_stream(dst + i, a);
+        st_stream(dst + i + stride, b);
+        st_stream(dst + i + 2 * stride, c);
+        st_stream(dst + i + 3 * stride, d);
+    }
+    for (; i < n16; i += stride) st_stream(dst + i, ld_stream(src + i));
+}
+
 // The library's bounded spin-wait on its own: one thread waits for *flag >=
 // target and raises FP4Q_FLAG_TIMEOUT if that does not happen within `limit`
 // polls, so that tests can watch a wait run out without any fault.
@@ -121,6 +140,17 @@ void launch_dequant(bool mx, const uint8_t* codes, const uint8_t* scales, const 
             dequant_kernel<float, false><<<g, kThreads, 0, s>>>(codes, scales, d_S, nb,
                                                                 static_cast<float*>(out));
     }
+}
+
+void launch_probe_copy(const void* src, void* dst, int64_t bytes, cudaStream_t s)
+{
+    const int64_t n16 = bytes / 16;
+    int64_t grid = (n16 + 4 * kThreads - 1) / (4 * kThreads);
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    probe_copy_kernel<<<(unsigned)grid, kThreads, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst),
+                                                           n16);
 }
 
 void launch_probe_wait(const unsigned* flag, unsigned target, unsigned limit, int32_t* d_status, cudaStream_t s)

@@ -73,6 +73,7 @@ void launch_mma_scale_layout(const uint8_t* s, int64_t rows, int64_t scols, uint
 void launch_dequant(bool mx, const uint8_t* codes, const uint8_t* scales, const float* d_S,
                     int64_t rows, int64_t cols, void* out, bool out_bf16, cudaStream_t s);
 
+void launch_probe_copy(const void* src, void* dst, int64_t bytes, cudaStream_t s);
 void launch_probe_wait(const unsigned* flag, unsigned target, unsigned limit, int32_t* d_status, cudaStream_t s);
 void launch_probe_e2m1(const float* r, uint8_t* out, int64_t n, cudaStream_t s);
 void launch_probe_e4m3(const float* v, uint8_t* out, int64_t n, cudaStream_t s);

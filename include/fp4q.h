@@ -494,6 +494,15 @@ fp4q_status fp4q_probe_e2m1(const float* r, uint8_t* out, int64_t n, fp4q_stream
 fp4q_status fp4q_probe_e4m3(const float* v, uint8_t* out, int64_t n, fp4q_stream_t stream);
 
 /*
+ * fp4q_probe_copy -- diagnostic with no counterpart in the papers: a plain
+ * streaming copy of `bytes` bytes (a multiple of 16, both pointers 16-byte
+ * aligned, not overlapping) with the library's 16-byte loads and stores, so
+ * that a benchmark can measure the copy bandwidth the library's own memory
+ * instructions reach (its HBM roofline peak).
+ */
+fp4q_status fp4q_probe_copy(const void* src, void* dst, int64_t bytes, fp4q_stream_t stream);
+
+/*
  * fp4q_probe_wait -- diagnostic with no counterpart in the papers: the
  * library's bounded spin-wait (the one the batch kernel and the one-launch
  * sweep use to wait for other thread blocks) run by one thread on its own.

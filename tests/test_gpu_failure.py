@@ -64,6 +64,20 @@ def test_bounded_wait_runs_out_and_the_context_survives():
     _assert_eq("codes", _np(r.codes), o["codes"])
 
 
+@pytest.mark.parametrize("nbytes", [0, 16, 48, 4096 + 16, 3 * 65536 + 208])
+def test_copy_probe_is_exact_and_stays_in_bounds(nbytes):
+    g = torch.Generator().manual_seed(nbytes)
+    src = torch.randint(0, 256, (nbytes,), dtype=torch.uint8, generator=g).to(DEV)
+    buf, dst = _guarded((nbytes,), torch.uint8)
+    fq.fp4q_probe_copy(src, dst)
+    torch.cuda.synchronize()
+    assert torch.equal(dst, src)
+    _intact("copy", buf, nbytes)
+    if nbytes >= 16:
+        with pytest.raises(fq.Fp4qError):           # not a multiple of 16 bytes
+            fq.fp4q_probe_copy(src[:8], dst[:8])
+
+
 @pytest.mark.parametrize("rows,cols", [(1, 32), (3, 96), (37, 288)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_guard_bytes_of_every_output(rows, cols, dtype):
