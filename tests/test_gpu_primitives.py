@@ -3,7 +3,10 @@
 The quantizer kernels round with the sm_100a conversions (E2M1 pairs and
 E4M3); these probes run the same device helpers over dense sets of inputs --
 every value within thousands of ulps of each rounding midpoint and grid point,
-plus millions of random bit patterns -- and compare with the CPU codecs.
+plus millions of random bit patterns -- and compare with the CPU codecs.  The
+exhaustive tests then cover every finite binary32 input: all 2^32 - 2^24 bit
+patterns for E2M1 (both signs) and all non-negative ones for E4M3 (the scale
+argument amax / (6 S) is never negative).
 """
 import numpy as np
 import pytest
@@ -68,3 +71,36 @@ def test_e4m3_conversion_matches_oracle():
     want = oracle.e4m3_encode_array(v)
     bad = np.nonzero(got != want)[0]
     assert bad.size == 0, f"{bad.size} mismatches; first v={v[bad[0]]!r} gpu={got[bad[0]]} oracle={want[bad[0]]}"
+
+
+CHUNK = 1 << 26
+FINITE_END = 0x7F800000          # first non-finite magnitude pattern (+Inf)
+
+
+def _exhaustive(probe, encode, negative: bool):
+    """Every finite pattern of one sign, CHUNK at a time: the inputs are made
+    on the device (an int32 range viewed as binary32) and on the host (the same
+    range as uint32), probed there, encoded by the oracle here, compared."""
+    out = torch.empty(CHUNK, dtype=torch.uint8, device=DEV)
+    base = 0x80000000 if negative else 0
+    signed_base = -(1 << 31) if negative else 0
+    for lo in range(0, FINITE_END, CHUNK):
+        hi = min(lo + CHUNK, FINITE_END)
+        vd = torch.arange(signed_base + lo, signed_base + hi, dtype=torch.int32, device=DEV).view(torch.float32)
+        probe(vd, out[:hi - lo])
+        got = out[:hi - lo].cpu().numpy()
+        v = np.arange(base + lo, base + hi, dtype=np.uint32).view(np.float32)
+        want = encode(v)
+        bad = np.nonzero(got != want)[0]
+        assert bad.size == 0, (f"{bad.size} mismatches in [{base + lo:#x}, {base + hi:#x}); first "
+                               f"bits={int(v[bad[0]:bad[0] + 1].view(np.uint32)[0]):#x} gpu={got[bad[0]]} "
+                               f"oracle={want[bad[0]]}")
+
+
+@pytest.mark.parametrize("negative", [False, True])
+def test_e2m1_conversion_every_finite_input(negative):
+    _exhaustive(fq.fp4q_probe_e2m1, oracle.e2m1_encode_array, negative)
+
+
+def test_e4m3_conversion_every_nonnegative_finite_input():
+    _exhaustive(fq.fp4q_probe_e4m3, oracle.e4m3_encode_array, False)
