@@ -310,30 +310,49 @@ def e2e_run(fq, model, steps, dev):
 
 # --------------------------------------------------------------------------- CPU baseline
 
-def cpu_sample_rows():
-    return 256
+CPU_SAMPLE_ROWS = 256          # rows per tensor of the calibration sample and the reference arm's step
 
 
-def cpu_baseline(seconds_hint=20.0):
-    """The oracle, as it stands, on a bounded sample of the workload: the first 256
-    rows of each of the 7 tensor shapes of one layer, NVFP4-MSE (absmax + sweep) and
-    MXFP4, all host cores (OpenMP)."""
+def _oracle_pass(rows):
+    """The oracle on the first `rows` rows (at most each tensor's own) of each of
+    the 7 tensor shapes of one layer: absmax + NVFP4-MSE sweep, and MXFP4.
+    Returns (elements, seconds); the inputs are made before the clock starts."""
     import oracle
     import synth
-    oracle.build()
-    rows = cpu_sample_rows()
     shapes = synth.llama3_8b_shapes()[:7]
-    xs = [synth.llama3_8b_tensor(i, rows, c, seed=7).float().numpy() for i, (_, _, c) in enumerate(shapes)]
+    xs = [synth.llama3_8b_tensor(i, min(rows, r), c, seed=7).float().numpy()
+          for i, (_, r, c) in enumerate(shapes)]
     n = sum(x.size for x in xs)
     t0 = time.perf_counter()
     for x in xs:
         g = oracle.global_absmax(x)
         oracle.nvfp4_quant(x, S=oracle.global_scale(g))
         oracle.mxfp4_quant(x)
-    dt = time.perf_counter() - t0
+    return n, time.perf_counter() - t0
+
+
+def cpu_baseline(target_s=12.0):
+    """The oracle, as it stands, on a bounded sample of the workload, all host
+    cores (OpenMP): a calibration pass on the first 256 rows of each of the 7
+    tensor shapes of one layer sets the row count of the timed pass so that it
+    takes about `target_s` seconds (never more rows than a tensor has)."""
+    import oracle
+    import synth
+    oracle.build()
+    n, dt = _oracle_pass(CPU_SAMPLE_ROWS)
+    rows = CPU_SAMPLE_ROWS
+    want = n * target_s / max(dt, 1e-3)               # elements for about target_s seconds
+    shapes = synth.llama3_8b_shapes()[:7]
+    full = max(r for _, r, _ in shapes)
+    grow = rows
+    while grow < full and sum(min(grow, r) * c for _, r, c in shapes) < want:
+        grow += 64
+    if grow > rows:
+        rows = grow
+        n, dt = _oracle_pass(rows)
     return {"value": 2.0 * n / dt / 1e9, "unit": "GB/s", "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": f"first {rows} rows of each of the 7 tensor shapes of one layer "
-                      f"({n} elements): absmax + NVFP4-MSE sweep + MXFP4, {dt:.2f}s",
+            "sample": f"first {rows} rows (at most each tensor's own) of each of the 7 tensor shapes of one "
+                      f"layer ({n} elements): absmax + NVFP4-MSE sweep + MXFP4, {dt:.2f}s",
             "elements_per_s": n / dt}
 
 
@@ -362,7 +381,7 @@ def run_reference(args):
     import oracle
     import synth
     oracle.build()
-    rows = 64
+    rows = CPU_SAMPLE_ROWS
     shapes = synth.llama3_8b_shapes()[:7]
     xs = [synth.llama3_8b_tensor(i, rows, c, seed=7).float().numpy() for i, (_, _, c) in enumerate(shapes)]
     n = sum(x.size for x in xs)
