@@ -1,5 +1,6 @@
 // api.cu -- the C ABI declared in include/fp4q.h: argument checks, then one
 // stream-ordered launch per call.  No allocation, no host synchronization.
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <map>
@@ -16,13 +17,16 @@ namespace fp4q {
 
 int sm_count()
 {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64];     // zero-initialized (static storage); any thread may fill a slot
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
-    if (dev < 64 && cached[dev] > 0) return cached[dev];
+    if (dev < 64) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    if (dev < 64) cached[dev] = n;
+    if (dev < 64) cached[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 
