@@ -19,9 +19,10 @@ tests/test_oracle_nvfp4.py and tests/test_oracle_mxfp4.py.  The optimality of
 the MXFP4 exponent window e0-1..e0+1 is not claimed by the pages and is
 "parity unpinned" beyond the defined computation.  ``scales_to_mma_layout``
 (the tiled scale layout read by Blackwell block-scaled GEMMs, a hardware
-interface the pages do not describe) is "parity unpinned" on the CPU: only its
-size and zero padding are checked there, and a library GEMM that reads the
-layout pins it on the GPU (tests/test_gpu_mma_layout.py).
+interface the pages do not describe) is pinned on the CPU against CUTLASS's
+hierarchical shape/stride definition of that layout, evaluated by a small
+independent layout-algebra routine in tests/test_oracle_mxfp4.py, and on the
+GPU by a library GEMM that reads it (tests/test_gpu_mma_layout.py).
 """
 from __future__ import annotations
 

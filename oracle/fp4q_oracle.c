@@ -37,8 +37,9 @@
  * codec sweeps against nearest-value search, the 126-value count, the window
  * ratios of Lemmas 4.1/4.3, brute force over all 126 scales, closed forms,
  * fp64 recomputation of losses, the dense Sylvester Hadamard matrix).
- * orc_scales_to_mma_layout is parity unpinned on the CPU (a hardware layout
- * the pages do not describe); a library GEMM reading it pins it on the GPU.
+ * orc_scales_to_mma_layout (a hardware layout the pages do not describe) is
+ * pinned against CUTLASS's shape/stride definition of the same layout, and
+ * by a library GEMM reading it on the GPU.
  */
 #include <math.h>
 #include <stdint.h>

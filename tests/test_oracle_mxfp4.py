@@ -158,9 +158,11 @@ def test_mxfp4_dequant_reproduces_reconstruction(orc):
 
 
 # ---------------------------------------------------------------- tiled scale layout
-# The layout itself is a hardware interface the pages do not describe ("parity
-# unpinned" on the CPU): a library GEMM pins it on the GPU.  Here: its size, that
-# every input byte lands exactly once, and that the padding is zero.
+# The layout is a hardware interface the pages do not describe.  Two pins: its
+# size, that every input byte lands exactly once and that the padding is zero
+# (here), and the position of every byte against the layout as CUTLASS defines
+# it (below, from its hierarchical shape/stride description); a library GEMM
+# reading it pins it once more on the GPU.
 
 @pytest.mark.parametrize("rows,scols", [(1, 1), (128, 4), (130, 6), (300, 257), (4096, 256)])
 def test_mma_layout_size_coverage_and_padding(orc, rows, scols):
@@ -171,3 +173,90 @@ def test_mma_layout_size_coverage_and_padding(orc, rows, scols):
     assert out.size == rt * ct * 512
     assert np.count_nonzero(out) == rows * scols                      # padding is zero
     assert sorted(out[out != 0].tolist()) == sorted(s.reshape(-1).tolist())
+
+
+# CUTLASS, include/cutlass/detail/sm100_blockscaled_layout.hpp: the scale-factor
+# atom of a K-major operand (Sm1xxBlockScaledBasicChunk::SfKMajorAtom) covers
+# 128 rows x 4 scales.  Its row mode has shape (32, 4) with strides (16, 4); its
+# K mode has shape (SFVecSize elements, 4 scales) with strides (0, 1) -- every
+# element of one scale's vector maps to the same byte.  tile_atom_to_shape_SFA
+# tiles the atom over (M, K) with Step<_2,_1>: atoms along K are adjacent.
+SF_ATOM = {"shape": ((32, 4), (16, 4)), "stride": ((16, 4), (0, 1))}   # SFVecSize = 16 (NVFP4)
+
+
+def _size(shape):
+    return int(np.prod([_size(s) for s in shape])) if isinstance(shape, tuple) else shape
+
+
+def _crd2idx(c, shape, stride):
+    """CuTe's coordinate -> index map: an integer coordinate of a tuple mode is
+    split colexicographically (first sub-mode fastest), then each part is mapped
+    by its sub-mode."""
+    if not isinstance(shape, tuple):
+        return c * stride
+    if isinstance(c, tuple):
+        return sum(_crd2idx(ci, si, di) for ci, si, di in zip(c, shape, stride))
+    idx = 0
+    for si, di in zip(shape, stride):
+        n = _size(si)
+        idx += _crd2idx(c % n, si, di)
+        c //= n
+    return idx
+
+
+def _cosize(shape, stride):
+    """One past the largest index the layout produces."""
+    last = tuple(_size(s) - 1 for s in shape)
+    return _crd2idx(last, shape, stride) + 1
+
+
+def _tile_to_shape(atom, target, order):
+    """Tile `atom` over `target` (each mode rounded up to whole atoms); the tile
+    counts of the modes are laid out one after another in the given order
+    (smallest step fastest), each tile cosize(atom) apart."""
+    a_shape, a_stride = atom["shape"], atom["stride"]
+    counts = [-(-t // _size(s)) for t, s in zip(target, a_shape)]
+    step = _cosize(a_shape, a_stride)
+    tile_stride = [0] * len(counts)
+    for m in sorted(range(len(counts)), key=lambda i: order[i]):
+        tile_stride[m] = step
+        step *= counts[m]
+    shape = tuple((a_shape[i], counts[i]) for i in range(len(counts)))
+    stride = tuple((a_stride[i], tile_stride[i]) for i in range(len(counts)))
+    return shape, stride, step
+
+
+@pytest.mark.parametrize("rows,scols", [(1, 1), (128, 4), (130, 6), (300, 37), (513, 65)])
+def test_mma_layout_matches_the_cutlass_layout_algebra(orc, rows, scols):
+    vec = 16
+    shape, stride, total = _tile_to_shape(SF_ATOM, (rows, scols * vec), order=(2, 1))
+    rng = np.random.default_rng(rows + 7 * scols)
+    s = rng.integers(1, 256, size=(rows, scols), dtype=np.uint8)
+    out = orc.scales_to_mma_layout(s)
+    assert out.size == total
+    want = np.zeros(total, dtype=np.uint8)
+    for r in range(rows):
+        for c in range(scols):
+            # every element k of scale c's vector addresses the same byte
+            offs = {_crd2idx((r, c * vec + j), shape, stride) for j in (0, vec // 2, vec - 1)}
+            assert len(offs) == 1
+            want[offs.pop()] = s[r, c]
+    np.testing.assert_array_equal(out, want)
+
+
+def test_cutlass_atom_constants_match_the_header():
+    """The atom numbers above against the CUTLASS header shipped in this image, when
+    one is there (a source file read as text)."""
+    import glob
+    import re
+    import site
+    paths = []
+    for root in site.getsitepackages():
+        paths += glob.glob(f"{root}/*/data/cutlass/include/cutlass/detail/sm100_blockscaled_layout.hpp")
+        paths += glob.glob(f"{root}/*/3rdparty/cutlass/include/cutlass/detail/sm100_blockscaled_layout.hpp")
+    if not paths:
+        pytest.skip("no CUTLASS header in this image")
+    text = re.sub(r"\s+", "", open(paths[0]).read())
+    assert "usingSfKMajorAtom=Layout<Shape<Shape<_32,_4>,Shape<Int<SFVecSize>,_4>>," in text
+    assert "Stride<Stride<_16,_4>,Stride<_0,_1>>>;" in text
+    assert "tile_to_shape(SfAtom{},make_shape(M,K),Step<_2,_1>{})" in text
