@@ -6,7 +6,9 @@ FP4 Quantization" (gist.science, arXiv 2509.23202), technical summary sec. 1
 grid; fused block Hadamard micro-rotation, orthogonal); TORQ summary (arXiv
 2605.19561) sec. 2.B (S-step maps the block maximum onto the largest code).
 The e0-1..e0+1 window itself has no optimality statement on the pages: beyond
-the defined computation it is parity unpinned.
+the defined computation it is parity unpinned; an fp64 brute force over twelve
+exponents finds the window's choice optimal in every block of two heavy-tailed
+synthetic weights (an observation, not a claim of the pages).
 """
 import numpy as np
 import pytest
@@ -140,6 +142,27 @@ def test_mxfp4_sweep_not_worse_than_centre(orc):
     inv = np.exp2(-e0.astype(np.float64)).astype(np.float32)[:, None]
     l0, _, _ = block_losses(xb, d, inv)
     assert np.all(out["loss"].reshape(-1) <= l0[:, 0] * (1 + 2 * RTOL_SUM32))
+
+
+@pytest.mark.parametrize("nu,scale,seed", [(4, 0.02, 31), (3, 0.015, 32)])
+def test_mxfp4_choice_is_the_best_of_all_exponents(orc, nu, scale, seed):
+    """fp64 brute force over twelve exponents around floor(log2 amax) (found here
+    with frexp, not with the oracle's centre rule): on heavy-tailed weights the
+    oracle's exponent attains the least loss of all of them in every block, so
+    the e0-1..e0+1 window and its centre are where the optimum lies."""
+    x = synth.t_weight(256, 1024, nu=nu, scale=scale, seed=seed).float().numpy()
+    out = orc.mxfp4_quant(x)
+    xb = x.reshape(-1, 32)
+    _, ex = np.frexp(np.abs(xb).max(axis=1).astype(np.float64))      # amax = m * 2^ex, m in [0.5, 1)
+    cand = (ex - 1)[:, None] + np.arange(-8, 4)[None, :]
+    d = np.exp2(cand.astype(np.float64)).astype(np.float32)
+    inv = np.exp2(-cand.astype(np.float64)).astype(np.float32)
+    loss64, _, _ = block_losses(xb, d, inv)
+    chosen = out["scales"].reshape(-1).astype(np.int64) - 127
+    assert np.all((chosen[:, None] == cand).any(axis=1))              # inside the brute-force range
+    k = np.argmax(cand == chosen[:, None], axis=1)
+    picked = loss64[np.arange(len(k)), k]
+    assert np.all(picked <= loss64.min(axis=1) * (1 + 2 * RTOL_SUM32) + 1e-37)
 
 
 def test_mxfp4_nonfinite_status(orc):
