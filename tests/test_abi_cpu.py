@@ -133,6 +133,55 @@ def test_dynamic_argument_errors_without_a_gpu(fq):
     assert call(nbytes=ws - 1) == fq.ERR_ARG
 
 
+def test_widening_entries_argument_errors_without_a_gpu(fq):
+    """FOCUS, the inverse rotation, GPTQ, the tiled scale layout and the copy
+    probe check their arguments before any CUDA call."""
+    lib = fq.load()
+    buf = ctypes.create_string_buffer(512)
+    p = ctypes.addressof(buf)
+    q = p + (-p % 16)
+    NV, MX = fq.NVFP4, fq.MXFP4
+    # FOCUS: format, sub-block size, shape, pointers, alignment
+    assert lib.fp4q_focus_quant(9, q, 1, 1, 16, q, q, q, 8, q, None, None, q, None) == fq.ERR_DTYPE
+    assert lib.fp4q_focus_quant(NV, q, 1, 1, 16, q, q, q, 32, q, None, None, q, None) == fq.ERR_ARG
+    assert lib.fp4q_focus_quant(NV, q, 1, 1, 16, q, q, q, 6, q, None, None, q, None) == fq.ERR_ARG
+    assert lib.fp4q_focus_quant(MX, q, 1, 1, 48, q, None, q, 8, q, None, None, q, None) == fq.ERR_SHAPE
+    assert lib.fp4q_focus_quant(NV, q, 1, 1, 16, q, None, q, 8, q, None, None, q, None) == fq.ERR_NULL
+    assert lib.fp4q_focus_quant(NV, q, 1, 1, 16, q, q, None, 8, q, None, None, q, None) == fq.ERR_NULL
+    assert lib.fp4q_focus_quant(NV, q, 1, 1, 16, q, q, q + 1, 8, q, None, None, q, None) == fq.ERR_ALIGN
+    assert lib.fp4q_focus_quant(MX, q, 1, 0, 32, None, None, None, 32, None, None, None, None, None) == fq.OK
+    # inverse rotation
+    assert lib.fp4q_mxfp4_unrotate(q, 4, 1, 32, q, q, None) == fq.ERR_DTYPE
+    assert lib.fp4q_mxfp4_unrotate(q, 1, 1, 16, q, q, None) == fq.ERR_SHAPE
+    assert lib.fp4q_mxfp4_unrotate(q, 1, 1, 32, None, q, None) == fq.ERR_NULL
+    assert lib.fp4q_mxfp4_unrotate(q, 1, 1, 32, q, q + 8, None) == fq.ERR_ALIGN
+    assert lib.fp4q_mxfp4_unrotate(None, 1, 0, 32, None, None, None) == fq.OK
+    # GPTQ: shape, pointers, workspace size
+    ws = fq.fp4q_gptq_workspace_bytes(4)
+    assert ws == 4 * 128 * 4 and fq.fp4q_gptq_workspace_bytes(0) == 0
+    assert lib.fp4q_nvfp4_gptq(q, 4, 24, q, q, q, q, q, None, q, ws, q, None) == fq.ERR_SHAPE
+    assert lib.fp4q_nvfp4_gptq(q, 4, 16, None, q, q, q, q, None, q, ws, q, None) == fq.ERR_NULL
+    assert lib.fp4q_nvfp4_gptq(q, 4, 16, q, q, q, q, q, None, None, ws, q, None) == fq.ERR_NULL
+    assert lib.fp4q_nvfp4_gptq(q, 4, 16, q, q, q, q, q, None, q + 4, ws, q, None) == fq.ERR_ALIGN
+    assert lib.fp4q_nvfp4_gptq(q, 4, 16, q, q, q, q, q, None, q, ws - 16, q, None) == fq.ERR_ARG
+    assert lib.fp4q_nvfp4_gptq(q, 4, (1 << 20) + 16, q, q, q, q, q, None, q, ws, q, None) == fq.ERR_SHAPE
+    # tiled scale layout: size arithmetic and checks
+    assert fq.fp4q_mma_scale_bytes(1, 1) == 512
+    assert fq.fp4q_mma_scale_bytes(129, 5) == 2 * 2 * 512
+    assert fq.fp4q_mma_scale_bytes(0, 7) == 0
+    assert fq.fp4q_mma_scale_bytes(-1, 4) == -1 and fq.fp4q_mma_scale_bytes(1 << 62, 4) == -1
+    assert lib.fp4q_scales_to_mma_layout(q, -1, 4, q, None) == fq.ERR_SHAPE
+    assert lib.fp4q_scales_to_mma_layout(None, 4, 4, q, None) == fq.ERR_NULL
+    assert lib.fp4q_scales_to_mma_layout(q, 4, 4, q + 4, None) == fq.ERR_ALIGN
+    assert lib.fp4q_scales_to_mma_layout(None, 0, 4, None, None) == fq.OK
+    # copy probe
+    assert lib.fp4q_probe_copy(q, q + 256, 24, None) == fq.ERR_SHAPE
+    assert lib.fp4q_probe_copy(q, q + 256, -16, None) == fq.ERR_SHAPE
+    assert lib.fp4q_probe_copy(None, q, 16, None) == fq.ERR_NULL
+    assert lib.fp4q_probe_copy(q + 8, q + 256, 16, None) == fq.ERR_ALIGN
+    assert lib.fp4q_probe_copy(None, None, 0, None) == fq.OK
+
+
 def test_binding_refuses_cpu_tensors(fq):
     w = torch.zeros((4, 32), dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
