@@ -67,6 +67,13 @@ def load_peaks():
 HBM_SPEC_GBS = 8000.0     # B200 HBM3e bandwidth as specified (context only)
 
 
+def l2_flush_buffer(dev):
+    """A buffer at least twice the device's L2 (and at least 512 MB): rewriting it
+    between timed launches leaves none of their inputs in L2."""
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or 0)
+    return torch.empty(max(512 << 20, 2 * l2), dtype=torch.uint8, device=dev)
+
+
 def copy_probe_gbs(fq, dev, nbytes=512 << 20, reps=10):
     """Copy bandwidth of the library's own 16-byte streaming loads and stores
     (`fp4q_probe_copy`, nbytes read + nbytes written, source larger than L2):
@@ -454,7 +461,8 @@ SINGLE_PATHS = {
 def run_single(args):
     """Time one kernel on one synthetic bf16 weight (`--shape RxC`), `--steps` launches
     after `--warmup`, each launch timed with CUDA events on its stream; between
-    launches a 512 MB buffer is rewritten so that no launch starts with its input in L2.
+    launches a buffer of twice the L2 (at least 512 MB) is rewritten so that no launch
+    starts with its input in L2.
     Prints one JSON line (not the benchmark line)."""
     import fp4_post_weight_grid_b200 as fq
     from fp4_post_weight_grid_b200 import build as fbuild
@@ -475,7 +483,7 @@ def run_single(args):
     deq = torch.empty_like(w)
     tiled = torch.empty(fq.fp4q_mma_scale_bytes(rows, cols // 16), dtype=torch.uint8, device=dev)
     coeffs = (1.0 + 0.25 * torch.rand((rows, cols // 8), device=dev)).to(torch.float16)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush = l2_flush_buffer(dev)
     fq.fp4q_global_absmax(w, amax)
     fq.fp4q_nvfp4_sweepmse(w, amax, codes, sc16, S, deq, None, st)
     fq.fp4q_mxfp4_quant(w, codes, sc32, None, None, st)
@@ -608,8 +616,8 @@ def run_configs(args):
     rotated MXFP4 28672 x 8192 (the whole-model pass is the benchmark line).
     Per record: the ABI sequence (global absmax + sweep, or the rotated MXFP4
     pass) timed with CUDA events, median of `--steps` launches after
-    `--warmup`, a 512 MB buffer rewritten between launches so that no launch
-    starts with its input in L2; algorithmic bytes and their fraction of the
+    `--warmup`, a buffer of twice the L2 (at least 512 MB) rewritten between
+    launches so that no launch starts with its input in L2; algorithmic bytes and their fraction of the
     measured HBM peak; parity with the oracle on sampled rows (all rows of
     the outlier matrix), element by element; the aggregate reconstruction MSE
     of those rows on both sides (fp64); the oracle's time on those rows."""
@@ -622,7 +630,7 @@ def run_configs(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     hbm_peak, peak_kind, _ = load_peaks()
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush = l2_flush_buffer(dev)
     stream = torch.cuda.current_stream()
     reps = max(args.steps, 5)
 
