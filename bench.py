@@ -320,10 +320,23 @@ def e2e_run(fq, model, steps, dev):
 CPU_SAMPLE_ROWS = 256          # rows per tensor of the calibration sample and the reference arm's step
 
 
-def _oracle_pass(rows):
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _oracle_pass(rows, threads=0):
     """The oracle on the first `rows` rows (at most each tensor's own) of each of
-    the 7 tensor shapes of one layer: absmax + NVFP4-MSE sweep, and MXFP4.
-    Returns (elements, seconds); the inputs are made before the clock starts."""
+    the 7 tensor shapes of one layer: absmax + NVFP4-MSE sweep, and MXFP4, on
+    `threads` OpenMP threads (0: all cores).  Returns (elements, seconds); the
+    inputs are made before the clock starts."""
     import oracle
     import synth
     shapes = synth.llama3_8b_shapes()[:7]
@@ -333,8 +346,8 @@ def _oracle_pass(rows):
     t0 = time.perf_counter()
     for x in xs:
         g = oracle.global_absmax(x)
-        oracle.nvfp4_quant(x, S=oracle.global_scale(g))
-        oracle.mxfp4_quant(x)
+        oracle.nvfp4_quant(x, S=oracle.global_scale(g), threads=threads)
+        oracle.mxfp4_quant(x, threads=threads)
     return n, time.perf_counter() - t0
 
 
@@ -357,10 +370,14 @@ def cpu_baseline(target_s=12.0):
     if grow > rows:
         rows = grow
         n, dt = _oracle_pass(rows)
+    n1, dt1 = _oracle_pass(64, threads=1)
     return {"value": 2.0 * n / dt / 1e9, "unit": "GB/s", "cores": oracle.max_threads(), "kind": "oracle",
             "sample": f"first {rows} rows (at most each tensor's own) of each of the 7 tensor shapes of one "
                       f"layer ({n} elements): absmax + NVFP4-MSE sweep + MXFP4, {dt:.2f}s",
-            "elements_per_s": n / dt}
+            "elements_per_s": n / dt, "cpu_model": _cpu_model(),
+            "single_thread": {"value": 2.0 * n1 / dt1 / 1e9, "unit": "GB/s", "elements_per_s": n1 / dt1,
+                              "sample": f"first 64 rows of each of the 7 tensor shapes ({n1} elements), "
+                                        f"1 thread, {dt1:.2f}s"}}
 
 
 def rank_seed(rank: int) -> int:

@@ -295,8 +295,8 @@ int orc_nvfp4_quant(const float* x, int64_t rows, int64_t cols, float S,
     int64_t nb = cols / bs, r;
     if (cols % bs) return 2;
 #ifdef _OPENMP
-    if (threads > 0) omp_set_num_threads(threads);
-#pragma omp parallel for schedule(static)
+    const int nt = threads > 0 ? threads : omp_get_max_threads();   /* this call only */
+#pragma omp parallel for schedule(static) num_threads(nt)
 #endif
     for (r = 0; r < rows; ++r) {
         int64_t b;
@@ -348,8 +348,8 @@ int orc_nvfp4_gptq(const float* x, int64_t rows, int64_t cols, const float* U, f
     int status = ORC_OK;
     if (cols % bs) return 2;
 #ifdef _OPENMP
-    if (threads > 0) omp_set_num_threads(threads);
-#pragma omp parallel for schedule(static)
+    const int nt = threads > 0 ? threads : omp_get_max_threads();   /* this call only */
+#pragma omp parallel for schedule(static) num_threads(nt)
 #endif
     for (r = 0; r < rows; ++r) {
         float* w = (float*)malloc((size_t)cols * sizeof(float));
@@ -398,8 +398,8 @@ int orc_nvfp4_bruteforce(const float* x, int64_t rows, int64_t cols, float S,
     int64_t nb = cols / bs, r;
     if (cols % bs) return 2;
 #ifdef _OPENMP
-    if (threads > 0) omp_set_num_threads(threads);
-#pragma omp parallel for schedule(static)
+    const int nt = threads > 0 ? threads : omp_get_max_threads();   /* this call only */
+#pragma omp parallel for schedule(static) num_threads(nt)
 #endif
     for (r = 0; r < rows; ++r) {
         int64_t b;
@@ -501,8 +501,8 @@ int orc_mxfp4_quant(const float* x, int64_t rows, int64_t cols, const uint32_t* 
     int status = ORC_OK;
     if (cols % bs) return 2;
 #ifdef _OPENMP
-    if (threads > 0) omp_set_num_threads(threads);
-#pragma omp parallel for schedule(static)
+    const int nt = threads > 0 ? threads : omp_get_max_threads();   /* this call only */
+#pragma omp parallel for schedule(static) num_threads(nt)
 #endif
     for (r = 0; r < rows; ++r) {
         int64_t b;
