@@ -67,6 +67,15 @@ def load_peaks():
 HBM_SPEC_GBS = 8000.0     # B200 HBM3e bandwidth as specified (context only)
 
 
+def tensor_sha256(t) -> str:
+    """SHA-256 of a tensor's (or array's) raw bytes in memory order, any dtype,
+    on any device (the bytes are copied to the host first)."""
+    import hashlib
+    if isinstance(t, torch.Tensor):
+        t = t.detach().contiguous().reshape(-1).view(torch.uint8).cpu().numpy()
+    return hashlib.sha256(memoryview(np.ascontiguousarray(t)).cast("B")).hexdigest()
+
+
 def l2_flush_buffer(dev):
     """A buffer at least twice the device's L2 (and at least 512 MB): rewriting it
     between timed launches leaves none of their inputs in L2."""
@@ -756,7 +765,11 @@ def run_configs(args):
                           "parity_rows": int(idx.size), "parity_bit_exact": bool(same),
                           "mse_gpu": mse_gpu, "mse_oracle": mse_orc,
                           "mse_rel_diff": abs(mse_gpu - mse_orc) / max(mse_orc, 1e-300),
-                          "oracle_s_on_rows": t_orc, "oracle_cores": oracle.max_threads()}), flush=True)
+                          "oracle_s_on_rows": t_orc, "oracle_cores": oracle.max_threads(),
+                          "input_sha256": {"w": tensor_sha256(w),
+                                           **({"importance": tensor_sha256(imp_np)} if make_imp else {}),
+                                           **({"sign_masks": tensor_sha256(masks_np)} if make_masks else {})}}),
+              flush=True)
         del w, deq, codes
         torch.cuda.empty_cache()
     return 0

@@ -1,0 +1,24 @@
+"""Host-side helpers of the benchmark, on the CPU."""
+import hashlib
+
+import numpy as np
+import torch
+
+import bench
+
+
+def test_tensor_sha256_hashes_the_raw_bytes_of_any_dtype():
+    g = torch.Generator().manual_seed(1)
+    x = torch.randn(3, 40, generator=g)
+    for t in (x, x.to(torch.bfloat16), x.to(torch.float16), (x * 100).to(torch.int32)):
+        raw = t.contiguous().numpy().tobytes() if t.dtype != torch.bfloat16 \
+            else t.view(torch.int16).numpy().tobytes()
+        assert bench.tensor_sha256(t) == hashlib.sha256(raw).hexdigest()
+    a = np.arange(10, dtype=np.uint32)
+    assert bench.tensor_sha256(a) == hashlib.sha256(a.tobytes()).hexdigest()
+    assert bench.tensor_sha256(x.t()) == hashlib.sha256(x.t().contiguous().numpy().tobytes()).hexdigest()
+
+
+def test_rank_seeds_differ_and_start_at_the_workload_seed():
+    assert bench.rank_seed(0) == 5
+    assert len({bench.rank_seed(r) for r in range(8)}) == 8
