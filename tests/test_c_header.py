@@ -40,6 +40,9 @@ int main(void)
     EXPECT(fp4q_nvfp4_gptq(f, 1, 16, f, f, u8, u8, f, NULL, p, 0, st, NULL), FP4Q_ERR_ARG);
     EXPECT(fp4q_scales_to_mma_layout(u8, -1, 4, u8, NULL), FP4Q_ERR_SHAPE);
     EXPECT(fp4q_dequant((fp4q_format)5, u8, u8, f, 1, 16, p, FP4Q_BF16, NULL), FP4Q_ERR_DTYPE);
+    EXPECT(fp4q_mxfp4_unrotate(p, FP4Q_BF16, 1, 48, (const uint32_t*)buf, p, NULL), FP4Q_ERR_SHAPE);
+    EXPECT(fp4q_probe_copy(p, buf + 1024, 24, NULL), FP4Q_ERR_SHAPE);
+    EXPECT(fp4q_probe_copy(buf + 8, buf + 1024, 32, NULL), FP4Q_ERR_ALIGN);
     if (fp4q_mma_scale_bytes(130, 6) != 2 * 2 * 512) { printf("FAIL mma bytes\n"); ++fails; }
     if (fp4q_gptq_workspace_bytes(5) != 8 * 128 * 4) { printf("FAIL gptq workspace\n"); ++fails; }
     printf(fails ? "failed\n" : "ok\n");
