@@ -850,7 +850,7 @@ def run_gptq(args):
 
 # --------------------------------------------------------------------------- main
 
-def main():
+def build_parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
@@ -876,7 +876,11 @@ def main():
     ap.add_argument("--chunk", type=int, default=128, help="weights per batch launch (at most 128)")
     ap.add_argument("--lag", type=int, default=0,
                     help="with --streams > 1: the MXFP4 pass of tensor t waits for the sweep of t - lag")
-    args = ap.parse_args()
+    return ap
+
+
+def main():
+    args = build_parser().parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.single:

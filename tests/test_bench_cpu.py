@@ -22,3 +22,22 @@ def test_tensor_sha256_hashes_the_raw_bytes_of_any_dtype():
 def test_rank_seeds_differ_and_start_at_the_workload_seed():
     assert bench.rank_seed(0) == 5
     assert len({bench.rank_seed(r) for r in range(8)}) == 8
+
+
+def test_profile_commands_use_existing_benchmark_options():
+    """Every `python bench.py ...` command quoted in profiles/ parses with the
+    benchmark's own options (the summaries must name commands that run)."""
+    import glob
+    import os
+    import re
+    import shlex
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmds = []
+    for path in glob.glob(os.path.join(root, "profiles", "*.md")):
+        text = open(path).read().replace("\\\n", " ")
+        cmds += [(path, m) for m in re.findall(r"python bench\.py([^`\n]*)", text)]
+    assert cmds, "no benchmark command found in profiles/"
+    parser = bench.build_parser()
+    for path, tail in cmds:
+        args = shlex.split(tail.split(">")[0])
+        parser.parse_args(args)          # SystemExit on an unknown option or kernel name
