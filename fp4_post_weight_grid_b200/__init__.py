@@ -17,6 +17,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import threading
 from typing import NamedTuple, Optional
 
 import torch
@@ -39,6 +40,7 @@ __all__ = [
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libfp4q.so")
 _lib = None
+_lib_lock = threading.Lock()
 
 OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_NONFINITE, ERR_CUDA, ERR_RANGE, ERR_ARG = range(9)
 F32, BF16 = 0, 1
@@ -82,10 +84,16 @@ def library_path() -> str:
 
 
 def load():
-    """Load libfp4q.so (raises if it has not been built)."""
-    global _lib
+    """Load libfp4q.so (raises if it has not been built).  Thread-safe: the
+    first caller loads it and declares the signatures, the others wait."""
     if _lib is not None:
         return _lib
+    with _lib_lock:
+        return _lib if _lib is not None else _load_locked()
+
+
+def _load_locked():
+    global _lib
     if not os.path.exists(_LIB_PATH):
         raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
                            "`python -m fp4_post_weight_grid_b200.build` (nvcc, sm_100a)")
