@@ -5,6 +5,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 
 #include <cuda_runtime.h>
@@ -33,18 +34,19 @@ int sm_count()
 int resident_blocks_per_sm(const void* kernel, int threads, size_t dyn_smem)
 {
     static std::mutex mu;
-    static std::map<std::pair<const void*, int>, int> cache;
+    static std::map<std::tuple<const void*, int, int, size_t>, int> cache;   // (kernel, device, threads, smem)
     int dev = 0;
     cudaGetDevice(&dev);
+    const auto key = std::make_tuple(kernel, dev, threads, dyn_smem);
     std::lock_guard<std::mutex> lock(mu);
-    auto it = cache.find({kernel, dev});
+    auto it = cache.find(key);
     if (it != cache.end()) return it->second;
     cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem);
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, dyn_smem) != cudaSuccess ||
         per_sm <= 0)
         per_sm = 1;
-    cache[{kernel, dev}] = per_sm;
+    cache[key] = per_sm;
     return per_sm;
 }
 
