@@ -43,11 +43,6 @@ WORKLOAD = "llama3-8b-shaped whole-model pass: 224 bf16 linear weights -> NVFP4-
 B_ABSMAX = 2.0
 B_NVFP4 = 2.0 + 0.5 + 1.0 / 16 + 2.0
 B_MXFP4 = 2.0 + 0.5 + 1.0 / 32 + 2.0
-# fp32 operations the definition needs per element and candidate:
-# r = x*inv, E2M1(r), y = q*d, e = x - y, e*e, L + e*e
-OPS_PER_ELEM_CAND = 6
-NVFP4_MSE_CANDIDATES = 11
-MXFP4_CANDIDATES = 3
 SM_FP32_LANES = 128
 
 
@@ -117,11 +112,12 @@ class ClockSampler:
     def __init__(self, gpu_id: str):
         self.gpu = gpu_id
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="fp4q_clocks_", suffix=".csv")
+        os.close(fd)
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                                           "-i", str(self.gpu), "-lms", "100"], stdout=self.fh,
@@ -154,6 +150,10 @@ class ClockSampler:
                 for n, v in zip(names, parts[5:9]):
                     if v.lower() == "active":
                         reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
@@ -276,6 +276,52 @@ class Model:
 
     def sweep_ms(self):
         return [a.elapsed_time(b) for a, b in self.events]
+
+
+PARITY_TENSORS = (0, 1, 2, 3, 4, 5, 6, 217, 218, 219, 220, 221, 222, 223)   # layers 0 and 31, all 7 shapes
+
+
+def step_parity(model, tensors=PARITY_TENSORS, rows_per_tensor=2):
+    """Outputs of the last timed step against the oracle, element by element, on
+    sampled rows of sampled tensors (outside the timed region): per tensor the
+    oracle's own global max over the whole weight gives S, which must equal the
+    S the sweep wrote; on rows 0 and rows-1 the NVFP4 codes, scales and bf16
+    reconstruction and the MXFP4 codes, scales and reconstruction must be
+    identical.  A schedule that let a sweep read its weight's maximum before
+    the MXFP4 pass had finished reducing it would show here."""
+    import oracle
+    oracle.build()
+    bad = []
+    checked = 0
+    for t in tensors:
+        if t >= len(model.w):
+            continue
+        w, o = model.w[t], model.out[t]
+        x_all = w.float().cpu().numpy()
+        rows = x_all.shape[0]
+        idx = np.array(sorted({0, rows - 1})[:rows_per_tensor])
+        x = np.ascontiguousarray(x_all[idx])
+        S_o = oracle.global_scale(oracle.global_absmax(x_all))
+        del x_all
+        nv = oracle.nvfp4_quant(x, S=S_o)
+        mx = oracle.mxfp4_quant(x)
+
+        def u16(tt):
+            return tt.detach().cpu().view(torch.int16).numpy().view(np.uint16)[idx]
+        ok = (np.float32(o["S"].item()) == np.float32(S_o)
+              and np.array_equal(o["nv_codes"].cpu().numpy()[idx], nv["codes"])
+              and np.array_equal(o["nv_scales"].cpu().numpy()[idx], nv["scales"])
+              and np.array_equal(u16(o["nv_deq"]), oracle.bf16_round(nv["y"]))
+              and np.array_equal(o["mx_codes"].cpu().numpy()[idx], mx["codes"])
+              and np.array_equal(o["mx_scales"].cpu().numpy()[idx], mx["scales"])
+              and np.array_equal(u16(o["mx_deq"]), oracle.bf16_round(mx["y"])))
+        checked += 1
+        if not ok:
+            bad.append(model.shapes[t][0])
+    return {"ok": not bad and checked > 0, "tensors_checked": checked, "rows_per_tensor": rows_per_tensor,
+            "mismatching": bad,
+            "what": "last timed step: S, NVFP4 codes/scales/bf16 reconstruction, MXFP4 codes/scales/bf16 "
+                    "reconstruction on rows 0 and rows-1 of layers 0 and 31, bit for bit against the oracle"}
 
 
 def e2e_run(fq, model, steps, dev):
@@ -443,26 +489,35 @@ def run_reference(args):
     return 0
 
 
-# --------------------------------------------------------------------------- measured DRAM traffic
-# dram__bytes_read.sum + dram__bytes_write.sum of one nvfp4_sweep_kernel (MSE, bf16)
-# launch on a 16384 x 8192 weight, per element, with the sources it was taken on
-# (profiles/nvfp4_sweep_mse_16384x8192.md).  Traffic grows in proportion to the
-# elements, so a launch of n elements moves about n times this.  Once the sources
-# differ the figure no longer describes the kernel and none is reported.
-NVFP4_TRAFFIC = {"bytes_per_element": (268480768 + 286225664) / (16384 * 8192),
+# --------------------------------------------------------------------------- measured counters
+# ncu counters of one nvfp4_sweep_kernel (MSE, bf16) launch on a 16384 x 8192
+# weight, per element, with the sources they were taken on
+# (profiles/nvfp4_sweep_mse_16384x8192.md): DRAM bytes (dram__bytes_read.sum +
+# dram__bytes_write.sum), executed warp instructions (smsp__inst_executed.sum)
+# and the issue-active fraction.  Traffic grows in proportion to the elements,
+# so a launch of n elements moves about n times the per-element figure.  Once
+# the sources differ the figures no longer describe the kernel and none is
+# reported.
+NVFP4_PROFILE = {"bytes_per_element": (268480768 + 286225664) / (16384 * 8192),
+                 "warp_inst_per_element": 225.4e6 / (16384 * 8192),
+                 "issue_active_pct": 79.2,
                  "sources": ("nvfp4.cu", "nvfp4_block.cuh", "screen.cuh", "device.cuh"),
                  "sha256": "eeaccfe992e1af1b0984c8a9ffe3cbcc1d13d088c6b8c2383109abd62a785fc2"}
 
 
-def measured_traffic_per_launch(elements_per_launch):
+def nvfp4_profile_current():
+    """NVFP4_PROFILE if the kernel's sources still hash to the profiled ones, else None."""
     import hashlib
     h = hashlib.sha256()
-    for f in NVFP4_TRAFFIC["sources"]:
+    for f in NVFP4_PROFILE["sources"]:
         with open(os.path.join(ROOT, "fp4_post_weight_grid_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
-    if h.hexdigest() != NVFP4_TRAFFIC["sha256"]:
-        return None
-    return NVFP4_TRAFFIC["bytes_per_element"] * elements_per_launch
+    return NVFP4_PROFILE if h.hexdigest() == NVFP4_PROFILE["sha256"] else None
+
+
+def measured_traffic_per_launch(elements_per_launch):
+    prof = nvfp4_profile_current()
+    return None if prof is None else prof["bytes_per_element"] * elements_per_launch
 
 
 # --------------------------------------------------------------------------- single-kernel mode
@@ -517,7 +572,7 @@ def run_single(args):
 
     def launch():
         if args.single == "absmax":
-            fq.fp4q_global_absmax(w, amax, stream)
+            fq.fp4q_global_absmax(w, amax, stream=stream)
         elif args.single == "nvfp4-mse":
             fq.fp4q_nvfp4_sweepmse(w, amax, codes, sc16, S, deq, None, st, stream)
         elif args.single == "nvfp4-wmse":
@@ -596,7 +651,7 @@ def run_act_latency(args):
         ws = torch.zeros(fq.fp4q_dynamic_workspace_bytes() // 4, dtype=torch.int32, device=dev)
 
         def two():
-            fq.fp4q_global_absmax(x, amax, stream)
+            fq.fp4q_global_absmax(x, amax, stream=stream)
             fq.fp4q_nvfp4_sweepmse(x, amax, codes, scales, S, deq, None, st, stream)
 
         def one():
@@ -635,18 +690,23 @@ def run_act_latency(args):
 
 # --------------------------------------------------------------------------- per-workload records
 
-def run_configs(args):
-    """One JSON record per small workload (not the benchmark line): the
-    outlier matrix (128 x 256 fp32, NVFP4-MSE), the q_proj-shaped 4096 x 4096
-    (NVFP4-MSE), the WMSE 11008 x 4096 with its importance vector and the
-    rotated MXFP4 28672 x 8192 (the whole-model pass is the benchmark line).
-    Per record: the ABI sequence (global absmax + sweep, or the rotated MXFP4
-    pass) timed with CUDA events, median of `--steps` launches after
-    `--warmup`, a buffer of twice the L2 (at least 512 MB) rewritten between
-    launches so that no launch starts with its input in L2; algorithmic bytes and their fraction of the
-    measured HBM peak; parity with the oracle on sampled rows (all rows of
-    the outlier matrix), element by element; the aggregate reconstruction MSE
-    of those rows on both sides (fp64); the oracle's time on those rows."""
+CONFIG_KEYS = ("cfg1", "cfg2", "cfg3", "cfg4", "focus")
+
+
+def config_records(steps, warmup, keys=CONFIG_KEYS):
+    """One record per smaller workload (not the benchmark line), yielded as it
+    is measured: the outlier matrix (128 x 256 fp32, NVFP4-MSE), the
+    q_proj-shaped 4096 x 4096 (NVFP4-MSE), the WMSE 11008 x 4096 with its
+    importance vector, the rotated MXFP4 28672 x 8192 and, for context, the
+    FOCUS forward quantizer on the q_proj shape.  Per record: the ABI sequence
+    (global absmax + sweep, or the rotated MXFP4 pass) timed with CUDA events,
+    median of `steps` launches after `warmup` (at least 3), a buffer of twice
+    the L2 (at least 512 MB) rewritten between launches so that no launch
+    starts with its input in L2; algorithmic bytes and their fraction of the
+    measured HBM peak; parity with the oracle on sampled rows (all rows of the
+    outlier matrix), element by element, the oracle's global scale coming from
+    its own maximum over the whole weight; the aggregate reconstruction MSE of
+    those rows on both sides (fp64); the oracle's time on those rows."""
     import fp4_post_weight_grid_b200 as fq
     from fp4_post_weight_grid_b200 import build as fbuild
     import oracle
@@ -658,11 +718,12 @@ def run_configs(args):
     hbm_peak, peak_kind, _ = load_peaks()
     flush = l2_flush_buffer(dev)
     stream = torch.cuda.current_stream()
-    reps = max(args.steps, 5)
+    reps = max(steps, 5)
+    warm = max(warmup, 3)
 
     def timed(fn):
         ts = []
-        for i in range(max(args.warmup, 3) + reps):
+        for i in range(warm + reps):
             flush.fill_(i & 0xFF)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
@@ -670,7 +731,7 @@ def run_configs(args):
             fn()
             b.record(stream)
             torch.cuda.synchronize()
-            if i >= max(args.warmup, 3):
+            if i >= warm:
                 ts.append(a.elapsed_time(b))
         return statistics.median(ts)
 
@@ -678,20 +739,21 @@ def run_configs(args):
         t = t.detach().cpu()
         return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
 
-    workloads = [
-        ("outliers 128x256 fp32, NVFP4-MSE", lambda: synth.small_outliers(), None, None, "nv"),
-        ("q_proj 4096x4096 bf16, NVFP4-MSE", lambda: synth.q_proj(4096, 4096, seed=2, device=dev), None, None,
-         "nv"),
-        ("WMSE 11008x4096 bf16, NVFP4-WMSE",
-         lambda: synth.t_weight(11008, 4096, nu=4, scale=0.02, seed=3, device=dev),
-         lambda: synth.importance_diag_xtx(cols=4096, tokens=2048, seed=3), None, "nv"),
-        ("MXFP4+Hadamard 28672x8192 bf16", lambda: synth.t_weight(28672, 8192, nu=3, scale=0.015, seed=4,
-                                                                 device=dev),
-         None, lambda: synth.sign_masks(8192, seed=4), "mx"),
-    ]
-    workloads.append(("FOCUS NVFP4 (sub-blocks of 8) 4096x4096 bf16",
-                      lambda: synth.q_proj(4096, 4096, seed=2, device=dev), None, None, "focus"))
-    for name, make_w, make_imp, make_masks, kind in workloads:
+    workloads = {
+        "cfg1": ("outliers 128x256 fp32, NVFP4-MSE", lambda: synth.small_outliers(), None, None, "nv"),
+        "cfg2": ("q_proj 4096x4096 bf16, NVFP4-MSE", lambda: synth.q_proj(4096, 4096, seed=2, device=dev), None,
+                 None, "nv"),
+        "cfg3": ("WMSE 11008x4096 bf16, NVFP4-WMSE",
+                 lambda: synth.t_weight(11008, 4096, nu=4, scale=0.02, seed=3, device=dev),
+                 lambda: synth.importance_diag_xtx(cols=4096, tokens=2048, seed=3), None, "nv"),
+        "cfg4": ("MXFP4+Hadamard 28672x8192 bf16",
+                 lambda: synth.t_weight(28672, 8192, nu=3, scale=0.015, seed=4, device=dev),
+                 None, lambda: synth.sign_masks(8192, seed=4), "mx"),
+        "focus": ("FOCUS NVFP4 (sub-blocks of 8) 4096x4096 bf16",
+                  lambda: synth.q_proj(4096, 4096, seed=2, device=dev), None, None, "focus"),
+    }
+    for key in keys:
+        name, make_w, make_imp, make_masks, kind = workloads[key]
         w = make_w().to(dev)
         rows, cols = w.shape
         n = rows * cols
@@ -709,7 +771,7 @@ def run_configs(args):
             scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
 
             def fn():
-                fq.fp4q_global_absmax(w, amax, stream)
+                fq.fp4q_global_absmax(w, amax, st, stream)
                 if imp is None:
                     fq.fp4q_nvfp4_sweepmse(w, amax, codes, scales, S, deq, None, st, stream)
                 else:
@@ -746,12 +808,15 @@ def run_configs(args):
         else:
             o = oracle.mxfp4_quant(x, sign_masks=masks_np)
         t_orc = time.perf_counter() - t0
+        del x_all
         deq_o = oracle.bf16_round(o["y"]) if w.dtype == torch.bfloat16 else o["y"]
         dg = bits(deq)[idx]
         same = (np.array_equal(bits(codes)[idx], o["codes"])
                 and (kind == "focus" or np.array_equal(bits(scales)[idx], o["scales"]))
                 and np.array_equal(dg.view(np.uint32) if dg.dtype == np.float32 else dg,
                                    deq_o.view(np.uint32) if deq_o.dtype == np.float32 else deq_o))
+        if kind == "nv":
+            same = same and bool(np.float32(S.item()) == np.float32(o["S"]))
         ref = o["rotated"] if kind == "mx" else x
         y_gpu = deq.float().cpu().numpy()[idx].astype(np.float64)
         y_orc = (deq_o.astype(np.uint32) << 16).view(np.float32).astype(np.float64) \
@@ -759,20 +824,43 @@ def run_configs(args):
         mse_gpu = float(np.mean((ref.astype(np.float64) - y_gpu) ** 2))
         mse_orc = float(np.mean((ref.astype(np.float64) - y_orc) ** 2))
         gbs = nbytes / (ms * 1e-3) / 1e9
-        print(json.dumps({"workload": name, "shape": [rows, cols], "ms": ms, "input_gbs": n * isz / (ms * 1e-3) / 1e9,
-                          "elements_per_s": n / (ms * 1e-3), "algorithmic_bytes": nbytes, "algorithmic_gbs": gbs,
-                          "hbm_frac": gbs / hbm_peak, "peak_kind": peak_kind, "status": int(st.item()),
-                          "parity_rows": int(idx.size), "parity_bit_exact": bool(same),
-                          "mse_gpu": mse_gpu, "mse_oracle": mse_orc,
-                          "mse_rel_diff": abs(mse_gpu - mse_orc) / max(mse_orc, 1e-300),
-                          "oracle_s_on_rows": t_orc, "oracle_cores": oracle.max_threads(),
-                          "input_sha256": {"w": tensor_sha256(w),
-                                           **({"importance": tensor_sha256(imp_np)} if make_imp else {}),
-                                           **({"sign_masks": tensor_sha256(masks_np)} if make_masks else {})}}),
-              flush=True)
+        rec = {"key": key, "workload": name, "shape": [rows, cols], "ms": ms,
+               "input_gbs": n * isz / (ms * 1e-3) / 1e9,
+               "elements_per_s": n / (ms * 1e-3), "algorithmic_bytes": nbytes, "algorithmic_gbs": gbs,
+               "hbm_frac": gbs / hbm_peak, "peak_kind": peak_kind, "status": int(st.item()),
+               "parity_rows": int(idx.size), "parity_bit_exact": bool(same),
+               "mse_gpu": mse_gpu, "mse_oracle": mse_orc,
+               "mse_rel_diff": abs(mse_gpu - mse_orc) / max(mse_orc, 1e-300),
+               "oracle_s_on_rows": t_orc, "oracle_cores": oracle.max_threads(),
+               "input_sha256": {"w": tensor_sha256(w),
+                                **({"importance": tensor_sha256(imp_np)} if make_imp else {}),
+                                **({"sign_masks": tensor_sha256(masks_np)} if make_masks else {})}}
         del w, deq, codes
         torch.cuda.empty_cache()
+        yield rec
+    del flush
+    torch.cuda.empty_cache()
+
+
+def run_configs(args):
+    """--configs: one JSON record per smaller workload (config_records)."""
+    for rec in config_records(args.steps, args.warmup):
+        print(json.dumps(rec), flush=True)
     return 0
+
+
+def per_config_summary(steps, warmup):
+    """The benchmark line's `per_config`: for the four smaller workloads, the
+    median time of their ABI sequence (L2 flushed between launches), the
+    algorithmic GB/s and HBM fraction, and bit-exact parity with the oracle on
+    sampled rows (config_records)."""
+    out = {}
+    for rec in config_records(steps, warmup, keys=("cfg1", "cfg2", "cfg3", "cfg4")):
+        out[rec["key"]] = {"workload": rec["workload"], "us_median": rec["ms"] * 1e3,
+                           "algorithmic_gbs": rec["algorithmic_gbs"], "hbm_frac": rec["hbm_frac"],
+                           "parity_bit_exact": rec["parity_bit_exact"], "parity_rows": rec["parity_rows"],
+                           "mse_rel_diff": rec["mse_rel_diff"], "status": rec["status"]}
+    return out
 
 
 # --------------------------------------------------------------------------- GPTQ
@@ -858,6 +946,8 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="leave out the per-workload records of the four smaller workloads")
     ap.add_argument("--configs", action="store_true",
                     help="one JSON record per small workload: time, bytes, roofline, parity, MSE, oracle time")
     ap.add_argument("--gptq", action="store_true",
@@ -968,46 +1058,49 @@ def main():
     bytes_in = 2.0 * n * world
     value = bytes_in / (ms * 1e-3) / 1e9
     clock_mhz = clk.get("sm_mhz") or sm_max
-    alu_peak = 148 * SM_FP32_LANES * clock_mhz * 1e6 / 1e12          # Tlane-op/s
     if args.mode == "batch":
         # the batch kernel: per-launch durations of the last timed step
         kname = "batch_kernel (NVFP4-MSE + MXFP4, bf16)"
         kern_ms = sum(ev[0].elapsed_time(ev[1]) for _, _, _, ev in model.chunks)
         kern_bytes = (B_NVFP4 + B_MXFP4) * n
-        kern_ops = OPS_PER_ELEM_CAND * (NVFP4_MSE_CANDIDATES + MXFP4_CANDIDATES) * n
         n_launch = len(model.chunks)
     else:
         # the NVFP4 sweep kernel: per-launch durations of the last timed step
         kname = "nvfp4_sweep_kernel (MSE, bf16)"
         kern_ms = sum(model.sweep_ms())
         kern_bytes = B_NVFP4 * n
-        kern_ops = OPS_PER_ELEM_CAND * NVFP4_MSE_CANDIDATES * n
         n_launch = len(model.shapes)
     kern_gbs = kern_bytes / (kern_ms * 1e-3) / 1e9
-    alu_achieved = kern_ops / (kern_ms * 1e-3) / 1e12
-    hbm_frac = kern_gbs / hbm_peak
-    alu_frac = alu_achieved / alu_peak
     per_launch = {"launches_per_step": n_launch, "mean_launch_ms": kern_ms / n_launch,
-                  "algorithmic_bytes_per_launch": kern_bytes / n_launch}
+                  "algorithmic_bytes_per_launch": kern_bytes / n_launch,
+                  "bytes_basis": "2 B bf16 in + 0.5 B codes + 1/16 B scale + 2 B bf16 reconstruction per element"}
     traffic = None
+    explain = {"note": "the kernel's time is set by its instruction issue rate, not by DRAM"}
     if args.mode != "batch":
         traffic = measured_traffic_per_launch(kern_bytes / n_launch / B_NVFP4)
-    if alu_frac > hbm_frac:
-        roof = {"bound": "alu", "achieved": alu_achieved, "peak": alu_peak, "unit": "Tlane-op/s",
-                "frac": alu_frac, "traffic": traffic, "kernel": kname,
-                "peak_basis": f"148 SMs x 128 fp32 lanes x {clock_mhz:.0f} MHz median SM clock",
-                "ops_basis": f"{OPS_PER_ELEM_CAND} fp32 operations per element and candidate of the definition",
-                "hbm": {"achieved": kern_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_frac,
-                        "peak_kind": peak_kind}, **per_launch}
-    else:
-        roof = {"bound": "hbm", "achieved": kern_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_frac,
-                "traffic": traffic, "kernel": kname, "peak_kind": peak_kind, **per_launch}
+        prof = nvfp4_profile_current()
+        issue_peak = 148 * 4 * 32 * clock_mhz * 1e6             # lane-instructions/s at one warp-instruction/clk/SMSP
+        if prof is not None:
+            ipe = prof["warp_inst_per_element"]
+            explain.update({
+                "warp_instructions_per_element": ipe,
+                "issue_active_pct_of_active_cycles": prof["issue_active_pct"],
+                "basis": "ncu smsp__inst_executed.sum and smsp__issue_active on one 16384x8192 launch "
+                         "(profiles/nvfp4_sweep_mse_16384x8192.md)",
+                "issue_bound_time_fraction": (n * ipe * 32 / issue_peak) / (kern_ms * 1e-3),
+                "issue_peak_lane_inst_per_s": issue_peak})
+        else:
+            explain["basis"] = "no ncu counters for the current sources"
+    roof = {"bound": "hbm", "achieved": kern_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": kern_gbs / hbm_peak,
+            "traffic": traffic, "kernel": kname, "peak_kind": peak_kind, **per_launch, "explain": explain}
     step_bytes = (B_NVFP4 + B_MXFP4) * n
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD, "tensors": len(model.shapes), "elements": n,
+                   "input_dtype": "bf16", "output_formats": "NVFP4 (E2M1 + E4M3 scales + fp32 S) and MXFP4 "
+                                                           "(E2M1 + E8M0 scales), bf16 reconstructions",
                    "input_bytes": 2 * n, "l2": "inputs 13.96 GB > 126 MB L2, no flush",
                    "parallelism": f"replicas x{world} (weak)", "graph": "one CUDA graph per step",
                    "mode": args.mode},
@@ -1022,6 +1115,9 @@ def main():
         "status": status,
     }
     if rank == 0:
+        par = step_parity(model)
+        line["parity"] = par["ok"]
+        line["parity_detail"] = par
         try:
             if args.e2e_steps < 1:
                 raise RuntimeError("skipped (--e2e-steps 0)")
@@ -1030,8 +1126,13 @@ def main():
                            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_dt * 1e3}
         except Exception as e:   # report, do not hide
             line["e2e"] = {"value": None, "unit": "GB/s", "error": repr(e)}
-        if not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline()
+        if world == 1 and not args.no_per_config:
+            del model, graph
+            torch.cuda.empty_cache()
+            line["per_config"] = per_config_summary(max(args.steps, 10), args.warmup)
+            graph = None
         print(json.dumps(line), flush=True)
     if dist is not None:
         del graph

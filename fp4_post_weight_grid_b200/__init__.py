@@ -106,7 +106,7 @@ def _load_locked():
     lib.fp4q_last_cuda_error.restype = ctypes.c_char_p
     lib.fp4q_last_cuda_error.argtypes = []
     sigs = {
-        "fp4q_global_absmax": [P, I, I64, P, P],
+        "fp4q_global_absmax": [P, I, I64, P, P, P],
         "fp4q_nvfp4_sweepmse": [P, I, I64, I64, P, P, P, P, P, P, P, P],
         "fp4q_nvfp4_sweepwmse": [P, I, I64, I64, P, P, P, P, P, P, P, P, P],
         "fp4q_mxfp4_quant": [P, I, I64, I64, P, P, P, P, P, P],
@@ -195,12 +195,16 @@ def _rc(w: torch.Tensor, block: int = 1):
 
 # --------------------------------------------------------------------------- C entry points
 
-def fp4q_global_absmax(x: torch.Tensor, d_amax: torch.Tensor, stream=None) -> None:
-    """d_amax[0] = max|x| (NaN if x holds a NaN).  ScaleSweep: S = max|x|/(256*6)."""
+def fp4q_global_absmax(x: torch.Tensor, d_amax: torch.Tensor, d_status: Optional[torch.Tensor] = None,
+                       stream=None) -> None:
+    """d_amax[0] = max|x| (NaN if x holds a NaN).  ScaleSweep: S = max|x|/(256*6).
+    With d_status (one int32 on the device) the call also ORs FLAG_NONFINITE or
+    FLAG_RANGE into it when that maximum cannot give a global scale."""
     dev = x.device
     xp = _dev(x, "x", device=dev)
     ap = _dev(d_amax, "d_amax", torch.float32, 1, dev)
-    _check(load().fp4q_global_absmax(xp, _wdtype(x), x.numel(), ap, _stream(stream)),
+    sp = _dev(d_status, "d_status", torch.int32, 1, dev)
+    _check(load().fp4q_global_absmax(xp, _wdtype(x), x.numel(), ap, sp, _stream(stream)),
            "fp4q_global_absmax")
 
 
@@ -545,7 +549,7 @@ def nvfp4_quantize(w: torch.Tensor, importance: Optional[torch.Tensor] = None, w
     scales = torch.empty((rows, cols // NVFP4_BLOCK), dtype=torch.uint8, **kw)
     deq = torch.empty_like(w) if with_deq else None
     loss = torch.empty((rows, cols // NVFP4_BLOCK), dtype=torch.float32, **kw) if with_loss else None
-    fp4q_global_absmax(w, amax, stream)
+    fp4q_global_absmax(w, amax, stream=stream)
     if importance is None:
         fp4q_nvfp4_sweepmse(w, amax, codes, scales, S, deq, loss, status, stream)
     else:
@@ -604,7 +608,7 @@ def nvfp4_gptq(w: torch.Tensor, U: torch.Tensor, with_deq=True, stream=None) -> 
     kw = dict(device=w.device)
     work = w.to(torch.float32).contiguous().clone()
     amax = torch.empty(1, dtype=torch.float32, **kw)
-    fp4q_global_absmax(work, amax, stream)
+    fp4q_global_absmax(work, amax, stream=stream)
     S = torch.empty(1, dtype=torch.float32, **kw)
     status = torch.zeros(1, dtype=torch.int32, **kw)
     codes = torch.empty((rows, cols // 2), dtype=torch.uint8, **kw)

@@ -9,6 +9,7 @@
 // block on the caller's float.
 #include "device.cuh"
 #include "launch.h"
+#include "nvfp4_block.cuh"
 
 namespace fp4q {
 
@@ -80,9 +81,20 @@ __global__ void __launch_bounds__(kThreads) absmax_kernel(const void* __restrict
     }
 }
 
+// After the reduction: flag a global max that the NVFP4 sweep cannot use
+// (NaN/Inf, or nonzero outside [2^-64, 2^64]), one warp, one word read.
+__global__ void __launch_bounds__(32) absmax_check_kernel(const float* __restrict__ d_amax,
+                                                          int32_t* __restrict__ d_status)
+{
+    if (threadIdx.x == 0) {
+        const int32_t flag = nvfp4_gmax_flag(*d_amax);
+        if (flag) atomicOr(d_status, flag);
+    }
+}
+
 }  // namespace
 
-void launch_absmax(const void* x, bool bf16, int64_t n, float* d_amax, cudaStream_t s)
+void launch_absmax(const void* x, bool bf16, int64_t n, float* d_amax, int32_t* d_status, cudaStream_t s)
 {
     cudaMemsetAsync(d_amax, 0, sizeof(float), s);
     if (n <= 0) return;
@@ -96,6 +108,7 @@ void launch_absmax(const void* x, bool bf16, int64_t n, float* d_amax, cudaStrea
         absmax_kernel<true><<<(unsigned)blocks, kThreads, 0, s>>>(x, n, out);
     else
         absmax_kernel<false><<<(unsigned)blocks, kThreads, 0, s>>>(x, n, out);
+    if (d_status) absmax_check_kernel<<<1, 32, 0, s>>>(d_amax, d_status);
 }
 
 }  // namespace fp4q

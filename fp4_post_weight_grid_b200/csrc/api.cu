@@ -124,13 +124,14 @@ const char* fp4q_status_string(fp4q_status status)
 const char* fp4q_last_cuda_error(void) { return g_last_cuda_error; }
 
 fp4q_status fp4q_global_absmax(const void* x, fp4q_dtype dt, int64_t n, float* d_amax,
-                               fp4q_stream_t stream)
+                               int32_t* d_status, fp4q_stream_t stream)
 {
     if (!valid_dtype(dt)) return FP4Q_ERR_DTYPE;
     if (n < 0) return FP4Q_ERR_SHAPE;
     if (!d_amax || (n > 0 && !x)) return FP4Q_ERR_NULL;
-    if ((x && !aligned(x, 16)) || !aligned(d_amax, 4)) return FP4Q_ERR_ALIGN;
-    fp4q::launch_absmax(x, dt == FP4Q_BF16, n, d_amax, reinterpret_cast<cudaStream_t>(stream));
+    if ((x && !aligned(x, 16)) || !aligned(d_amax, 4) || (d_status && !aligned(d_status, 4)))
+        return FP4Q_ERR_ALIGN;
+    fp4q::launch_absmax(x, dt == FP4Q_BF16, n, d_amax, d_status, reinterpret_cast<cudaStream_t>(stream));
     return after_launch();
 }
 

@@ -30,7 +30,9 @@ inline int64_t resident_grid(Kernel kernel, int threads, size_t dyn_smem, int64_
     return g < 1 ? 1 : g;
 }
 
-void launch_absmax(const void* x, bool bf16, int64_t n, float* d_amax, cudaStream_t s);
+// Global max|x| into *d_amax; with d_status != nullptr a one-warp kernel then
+// flags a non-finite or out-of-range result.
+void launch_absmax(const void* x, bool bf16, int64_t n, float* d_amax, int32_t* d_status, cudaStream_t s);
 
 // NVFP4 ScaleSweep: importance == nullptr selects MSE (window -3..+7), otherwise
 // WMSE (window -8..+7).

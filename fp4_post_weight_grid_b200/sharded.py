@@ -64,7 +64,7 @@ def nvfp4_quantize_row_shard(w_shard: torch.Tensor, group=None, importance: Opti
 
     def local_absmax():
         amax = torch.empty(1, dtype=torch.float32, **kw)
-        fp4q_global_absmax(w_shard, amax, stream)
+        fp4q_global_absmax(w_shard, amax, stream=stream)
         return amax
 
     def all_reduce_max(amax):

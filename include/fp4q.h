@@ -114,11 +114,18 @@ const char* fp4q_last_cuda_error(void);
  *           every thread block merges its maximum with an atomic max on the
  *           bit pattern).  A NaN anywhere makes *d_amax a NaN; an Inf makes it
  *           +Inf.  n == 0 leaves *d_amax = 0.
+ *   d_status  device int32 or NULL.  When given, a one-warp kernel enqueued
+ *           after the reduction reads the final *d_amax and ORs
+ *           FP4Q_FLAG_NONFINITE into *d_status if it is a NaN or an Inf, or
+ *           FP4Q_FLAG_RANGE if it is nonzero and outside [2^-64, 2^64] (the
+ *           range inside which the NVFP4 sweep accepts a global max), so a
+ *           caller of this call alone learns whether the global scale is
+ *           usable.  NULL skips that check (the sweep performs it anyway).
  * Errors: FP4Q_ERR_NULL, FP4Q_ERR_SHAPE (n < 0), FP4Q_ERR_DTYPE,
  * FP4Q_ERR_ALIGN, FP4Q_ERR_CUDA.
  */
 fp4q_status fp4q_global_absmax(const void* x, fp4q_dtype dt, int64_t n, float* d_amax,
-                               fp4q_stream_t stream);
+                               int32_t* d_status, fp4q_stream_t stream);
 
 /*
  * fp4q_nvfp4_sweepmse -- NVFP4 ScaleSweep with the MSE objective.

@@ -70,8 +70,11 @@ def test_argument_errors_without_a_gpu(fq):
     assert lib.fp4q_mxfp4_quant_hadamard(p16, 1, 1, 32, None, p16, p16, None, None, p16, None) == fq.ERR_NULL
     assert lib.fp4q_dequant(5, p16, p16, p16, 1, 16, p16, 1, None) == fq.ERR_DTYPE
     assert lib.fp4q_dequant(0, p16, p16, None, 1, 16, p16, 1, None) == fq.ERR_NULL
-    assert lib.fp4q_global_absmax(p16, 1, -5, p16, None) == fq.ERR_SHAPE
-    assert lib.fp4q_global_absmax(p16 + 4, 1, 5, p16, None) == fq.ERR_ALIGN
+    assert lib.fp4q_global_absmax(p16, 1, -5, p16, None, None) == fq.ERR_SHAPE
+    assert lib.fp4q_global_absmax(p16 + 4, 1, 5, p16, None, None) == fq.ERR_ALIGN
+    assert lib.fp4q_global_absmax(p16, 1, 5, p16, p16 + 2, None) == fq.ERR_ALIGN
+    assert lib.fp4q_global_absmax(p16, 7, 5, p16, p16, None) == fq.ERR_DTYPE
+    assert lib.fp4q_global_absmax(p16, 1, 5, None, p16, None) == fq.ERR_NULL
     # empty tensors are valid and touch nothing
     assert lib.fp4q_nvfp4_sweepmse(None, 1, 0, 16, None, None, None, None, None, None, None, None) == fq.OK
     assert lib.fp4q_mxfp4_quant(None, 0, 5, 0, None, None, None, None, None, None) == fq.OK

@@ -28,7 +28,8 @@ int main(void)
     int32_t* st = (int32_t*)buf;
     if (fp4q_version() < 10000) { printf("FAIL version\n"); ++fails; }
     if (strcmp(fp4q_status_string(FP4Q_OK), "ok") != 0) { printf("FAIL status string\n"); ++fails; }
-    EXPECT(fp4q_global_absmax(p, FP4Q_BF16, -1, f, NULL), FP4Q_ERR_SHAPE);
+    EXPECT(fp4q_global_absmax(p, FP4Q_BF16, -1, f, NULL, NULL), FP4Q_ERR_SHAPE);
+    EXPECT(fp4q_global_absmax(p, FP4Q_BF16, 8, f, (int32_t*)(buf + 2), NULL), FP4Q_ERR_ALIGN);
     EXPECT(fp4q_nvfp4_sweepmse(p, (fp4q_dtype)7, 1, 16, f, u8, u8, f, NULL, NULL, st, NULL), FP4Q_ERR_DTYPE);
     EXPECT(fp4q_nvfp4_sweepmse(p, FP4Q_BF16, 1, 24, f, u8, u8, f, NULL, NULL, st, NULL), FP4Q_ERR_SHAPE);
     EXPECT(fp4q_nvfp4_sweepwmse(p, FP4Q_BF16, 1, 16, f, NULL, u8, u8, f, NULL, NULL, st, NULL), FP4Q_ERR_NULL);

@@ -98,6 +98,38 @@ def test_absmax_tails_and_dtypes():
             assert _np(a)[0] == oracle.global_absmax(x.float().numpy())
 
 
+def test_absmax_status_word_flags_unusable_maxima():
+    """fp4q_global_absmax alone reports, through its status word, a maximum that
+    cannot give a global scale (ScaleSweep summary, "Metodologia" sec. 2:
+    S = max|x| / 1536): NaN/Inf, or nonzero outside [2^-64, 2^64]."""
+    cases = [
+        (np.array([1.0, np.nan, 2.0] + [0.5] * 13, np.float32), fq.FLAG_NONFINITE),
+        (np.array([1.0, -np.inf] + [0.5] * 14, np.float32), fq.FLAG_NONFINITE),
+        (np.array([3.0 * 2.0 ** 70] + [1.0] * 15, np.float32), fq.FLAG_RANGE),
+        (np.array([2.0 ** -70] * 16, np.float32), fq.FLAG_RANGE),
+        (np.zeros(16, np.float32), 0),
+        (np.array([2.0 ** -64] + [0.0] * 15, np.float32), 0),
+        (np.array([2.0 ** 64] + [0.0] * 15, np.float32), 0),
+        (np.array([0.75] * 16, np.float32), 0),
+    ]
+    for x, want in cases:
+        for dt in (torch.float32, torch.bfloat16):
+            xt = torch.from_numpy(x).to(dt)      # every value above is exact in bf16
+            a = torch.empty(1, dtype=torch.float32, device=DEV)
+            st = torch.zeros(1, dtype=torch.int32, device=DEV)
+            fq.fp4q_global_absmax(xt.to(DEV), a, st)
+            torch.cuda.synchronize()
+            assert int(st.item()) == want, (x[:3], dt, int(st.item()))
+            got = _np(a)[0]
+            ref = oracle.global_absmax(xt.float().numpy())
+            assert (np.isnan(got) and np.isnan(ref)) or got == ref
+    # NULL status word: no flag anywhere, the maximum is still written
+    a = torch.empty(1, dtype=torch.float32, device=DEV)
+    fq.fp4q_global_absmax(torch.from_numpy(cases[0][0]).to(DEV), a)
+    torch.cuda.synchronize()
+    assert np.isnan(_np(a)[0])
+
+
 def test_stream_and_graph_capture_reproduce_eager():
     w = synth.q_proj(512, 1024, seed=45).to(DEV)
     eager = fq.nvfp4_quantize(w)
