@@ -466,8 +466,14 @@ fp4q_status fp4q_quantize_batch(const fp4q_batch_tensor* tensors, int32_t n, fp4
  *             returns FP4Q_ERR_ARG before anything is enqueued.
  * Other arguments, results and errors as fp4q_quantize_batch.
  * The first call on a device looks up the scratch's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  The scratch is zeroed, stream-ordered, at the
+ * (cudaGetSymbolAddress, with that device current) and keeps it for the rest
+ * of the process; make that first call before any stream capture.  Under lazy
+ * module loading that first call is also what loads the library's device code
+ * on that device, which is when the runtime places the scratch (the one
+ * allocation involved, done by the runtime, once).  The kept address belongs
+ * to the device's current context: after cudaDeviceReset on that device it is
+ * stale and this entry point must not be called again in the process.  The
+ * scratch is zeroed, stream-ordered, at the
  * start of every call, but it is shared by all calls on a device: calls whose
  * launches overlap on the GPU (different streams without ordering between
  * them) race on it and give wrong results.

@@ -672,9 +672,10 @@ int orc_focus_quant(int fmt, const float* x, int64_t rows, int64_t cols, const u
  * after the other, the column tiles of one row tile together.  A tile is 512
  * bytes: 32 lines of 16 bytes, line j holding rows j, j+32, j+64, j+96 of the
  * tile, 4 scale bytes each.  This is a hardware interface, not part of the
- * method; the pages do not describe it.  Parity pinned on the GPU only: a
- * library block-scaled GEMM reads this layout in tests/test_gpu_mma_layout.py;
- * on the CPU only its shape and its zero padding are checked. */
+ * method; the pages do not describe it.  Parity pinned on the CPU against
+ * CUTLASS's shape/stride definition of the same layout (byte for byte, ragged
+ * shapes; tests/test_oracle_mxfp4.py) and on the GPU by a library
+ * block-scaled GEMM that reads it (tests/test_gpu_mma_layout.py). */
 int64_t orc_mma_scale_bytes(int64_t rows, int64_t scols)
 {
     return ((rows + 127) / 128) * ((scols + 3) / 4) * 512;
