@@ -22,6 +22,8 @@
 // and v^2 come from shared-memory tables built once per global scale.
 #pragma once
 
+#include <type_traits>
+
 #include "device.cuh"
 #include "screen.cuh"
 
@@ -200,7 +202,17 @@ __device__ __forceinline__ void nvfp4_block(const NvTables& tb, const NvScale& c
     // term are symmetric in the sign, so the losses equal those of |x|.
     float x[16];
     uint32_t abits;
-    load_block_amax<16>(src, x, abits);
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        // the global max was checked finite, so no NaN can reach this block:
+        // a float max of |x| is the block maximum
+        load_block<16>(src, x);
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(x[i]));
+        abits = __float_as_uint(m);
+    } else {
+        load_block_amax<16>(src, x, abits);
+    }
     const float amax = __uint_as_float(abits);
     float alpha2;
     float wt[16];

@@ -27,14 +27,10 @@
 //    (32-term for MXFP4) sequential sums round at most n+2 times relative to
 //    their terms; (c) d^2 = v^2 S^2 (1+delta)^2.  The constants K1 = 128,
 //    K2 = 16, K3 = 64 are about twice what (a)-(c) need for 32-term blocks.
-//    Let M = min lam (candidate w).  The winner's true loss is at most U, the
-//    root of U = M + D(U), and a candidate k can only win if
-//    lam_k - D(lam_k) <= U; using sqrt(z) <= (z/sqrt(U) + sqrt(U))/2 this holds
-//    whenever lam_k <= T = (U + u*K2*alpha*sqrt(U)/2 + K3*u^2*alpha^2 + tau) /
-//    (1 - u*K1 - u*K2*alpha/(2*sqrt(U))), so every candidate with lam_k > T is
-//    excluded.  survivor_threshold evaluates an upper bound of T with
-//    approximate square roots and reciprocals, each widened, and widens the
-//    result by another 2^-10 relative, far more than their errors.
+//    Let M = min lam.  Bounding the square-root term linearly (see
+//    survivor_threshold) gives a threshold T = (M + 2b) / (1 - a)^2 above
+//    which no candidate can hold the exact minimum, so every candidate with
+//    lam_k > T is excluded.
 // 3. Verify.  The survivors (the screening minimum always survives; on
 //    typical weights about 1.002 per block) are evaluated with the exact
 //    definition in ascending order and the first minimum wins.  With a single
@@ -54,54 +50,29 @@ constexpr float kK1 = 128.0f;
 constexpr float kK2 = 16.0f;
 constexpr float kK3 = 64.0f;
 
-// Approximate square root, reciprocal square root and reciprocal (flush-to-zero
-// forms, single hardware instructions); callers widen every result so that the
-// threshold only grows, and pass normal inputs.
-__device__ __forceinline__ float sqrt_approx(float x)
-{
-    float r;
-    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
-}
-
-__device__ __forceinline__ float rsqrt_approx(float x)
-{
-    float r;
-    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
-}
-
-__device__ __forceinline__ float rcp_approx(float x)
-{
-    float r;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
-}
-
 // Largest screened loss that can still belong to the exact winner.
 //   M      minimum screened loss lam over the candidates
 //   alpha2 an upper bound of ||x||^2 / S^2 (or of the weighted norm); the
 //          bound D grows with alpha, so any upper bound keeps it valid
 //   tau    absolute allowance, in units of S^2 (at least 2^-120)
-// With a = 1 - u*K1, b = u*K2*alpha and c >= M + K3*u^2*alpha^2 + tau:
-//   sqrt(U) = (b + sqrt(b^2 + 4*a*c')) / (2a) <= (b + sqrt(c)) / a =: s (c' <= c),
-// and 1/s <= min(rho, 1/b) with rho >= 1/sqrt(c).  Any t > 0 may stand for
-// sqrt(U) in the bound sqrt(z) <= (z/t + t)/2; with t = s,
-//   T = (s^2 + b*s/2 + K3*u^2*alpha^2 + tau) / (1 - u*K1 - min(b*rho/2, 1/2)),
-// whose denominator is at least 1/2 - u*K1 (every candidate is kept if a NaN
-// makes it fail the test below).
+// The square-root term is bounded linearly: sqrt(z) <= (z/(g alpha) + g alpha)/2
+// for g = 2^-8, so D(z) <= a z + b with
+//   a = u (K1 + K2 / (2g)),   b = u K2 g alpha^2 / 2 + K3 u^2 alpha^2 + tau.
+// The winner's true loss is at most that of the screening minimum, which is at
+// most U = (M + b) / (1 - a).  A candidate k can only win if l_k <= U, and
+// l_k >= lam_k - a max(l_k, lam_k) - b, so it needs lam_k <= (U + b) / (1 - a)
+// <= (M + 2b) / (1 - a)^2.  That threshold is widened by another 2^-10
+// relative (and b by 2^-16), far more than the two roundings of its
+// evaluation; a = 2176 u, so it admits candidates within about 0.12% of the
+// minimum on a typical block.
 __device__ __forceinline__ float survivor_threshold(float M, float alpha2, float tau)
 {
-    const float alpha = sqrt_approx(fmaxf(alpha2, 0x1p-126f)) * (1.0f + 0x1p-16f);
-    const float hb = (0.5f * kU * kK2) * alpha;                    // b/2
-    const float k3 = (kK3 * kU * kU) * alpha2;
-    const float c = (M + k3 + tau) * (1.0f + 0x1p-16f);
-    const float rho = rsqrt_approx(c) * (1.0f + 0x1p-16f);         // >= 1/sqrt(c)
-    const float s = (2.0f * hb + c * rho) * (1.0f + 0x1p-15f);    // >= sqrt(U)
-    const float den = (1.0f - kU * kK1) - fminf(hb * rho, 0.5f);
-    if (!(den > 0.25f)) return __int_as_float(0x7F800000);          // keep all
-    const float T = (s * s + hb * s + k3 + tau) * rcp_approx(den);
-    return T * (1.0f + 0x1p-10f);
+    constexpr float kG = 0x1p-8f;
+    constexpr float kA = kU * (kK1 + kK2 / (2.0f * kG));
+    constexpr float kB = 0.5f * kU * kK2 * kG + kK3 * kU * kU;
+    constexpr float kC = (1.0f + 0x1p-10f) / ((1.0f - kA) * (1.0f - kA));
+    const float b = __fmaf_rn(alpha2, kB * (1.0f + 0x1p-16f), tau);
+    return __fmaf_rn(2.0f, b, M) * kC;
 }
 
 // f16x2 of the E2M1 rounding of (lo, hi); the code byte stays in a PTX .b8.

@@ -49,7 +49,7 @@ def _screen(orc, x, S, lo, hi, w=None):
         alpha2 = (wb * (a * invS).astype(np.float64) ** 2).sum(1) * (1 + 2 ** -16)
         tau = ((2.0 ** -70 / float(S)) ** 2 + 2.0 ** -120) * (1 + wb.max(1))
     M = lam.min(1)
-    T = np.array([float(kernel_threshold(M[i], alpha2[i], tau[i], e=0.0)) for i in range(len(M))])
+    T = np.array([float(kernel_threshold(M[i], alpha2[i], tau[i])) for i in range(len(M))])
     return cand, lam <= T[:, None]
 
 
