@@ -15,17 +15,22 @@
 // in ascending j, whether they are applied column by column or block by
 // block; so the blocked algorithm below writes exactly the bytes of the plain
 // sequential one.  Per block of 128 columns:
-//   gptq_block_kernel   4 threads per row, each holding two 16-column groups
-//                       of the block in registers, U's diagonal block in
-//                       shared memory: the sweep at every group start, the
-//                       column quantization by the group's owner, the error
-//                       broadcast by a warp shuffle, the in-block updates;
-//                       the scaled errors go to a workspace E;
-//   gptq_update_kernel  the trailing update of the columns after the block,
-//                       a 128 x 128 output tile per thread block (8 x 8 per
-//                       thread), each output a chain of exact fused
-//                       multiply-adds over the block's columns in ascending
-//                       order.
+//   in-block GPTQ   4 threads per row, each holding two 16-column groups of
+//                   the block in registers, U's diagonal block in shared
+//                   memory: the sweep at every group start, the column
+//                   quantization by the group's owner, the error broadcast by
+//                   a warp shuffle, the in-block updates; the scaled errors go
+//                   to a workspace E (two buffers, alternating per block);
+//   trailing update the columns after a block, a 128 x 128 output tile per
+//                   thread block (8 x 8 per thread), each output a chain of
+//                   exact fused multiply-adds over the block's columns in
+//                   ascending order.
+// The in-block part has only the rows as parallelism (four threads per row
+// along a sequential chain of columns), so on its own it leaves most of the
+// GPU idle.  Block J's in-block part therefore runs in one launch with the
+// bulk of block J-1's trailing update (the columns from block J+1 on), which
+// fills the rest of the GPU; a small launch then applies block J's errors to
+// block J+1's columns before block J+1's step.
 // The trailing update is a dense contraction, but it runs on the CUDA cores:
 // its definition is a chain of single-rounding fused multiply-adds in a fixed
 // order, which a tensor-core accumulation (another precision and order) would
@@ -67,29 +72,29 @@ __device__ __forceinline__ void gptq_update16(float (&x)[16], float e, const flo
 // columns with w_c = fma(-e_j, U[j][c], w_c), so each value sees the updates
 // in ascending j.  Eight rows share a warp, so the owner's serial work runs
 // on eight lanes at once.
-__global__ void __launch_bounds__(kThreadsA)
-gptq_block_kernel(const float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0, int bw,
-                  const float* __restrict__ U, const float* __restrict__ d_amax, uint8_t* __restrict__ codes,
-                  uint8_t* __restrict__ scales, float* __restrict__ d_S, float* __restrict__ deq,
-                  float* __restrict__ Et, int64_t ldE, int32_t* __restrict__ d_status, float neg_zero)
+__device__ __forceinline__ void gptq_block_body(int64_t cta, float* Us, NvTables& tb,
+                                                const float* __restrict__ w, int64_t rows, int64_t cols,
+                                                int64_t j0, int bw, const float* __restrict__ U,
+                                                const float* __restrict__ d_amax, uint8_t* __restrict__ codes,
+                                                uint8_t* __restrict__ scales, float* __restrict__ d_S,
+                                                float* __restrict__ deq, float* __restrict__ Et, int64_t ldE,
+                                                int32_t* __restrict__ d_status, float neg_zero)
 {
-    extern __shared__ __align__(16) float Us[];      // [bw][bw]: U's diagonal block
-    __shared__ NvTables tb;
     const float gmax = __ldg(d_amax);
     const int32_t flag = nvfp4_gmax_flag(gmax);
     if (flag) {
-        if (blockIdx.x == 0 && threadIdx.x == 0 && j0 == 0) atomicOr(d_status, flag);
+        if (cta == 0 && threadIdx.x == 0 && j0 == 0) atomicOr(d_status, flag);
         return;
     }
     const NvScale c = nvfp4_scale(gmax);
-    if (blockIdx.x == 0 && threadIdx.x == 0 && j0 == 0) *d_S = c.S;
+    if (cta == 0 && threadIdx.x == 0 && j0 == 0) *d_S = c.S;
     for (int i = threadIdx.x; i < bw * bw; i += kThreadsA)
         Us[i] = __ldg(U + (j0 + i / bw) * cols + j0 + i % bw);
     nvfp4_tables(tb, c.S);                           // synchronises: U's block is in place too
 
     const int lane = threadIdx.x & (kLanes - 1);
     const int src0 = (threadIdx.x & 31) & ~(kLanes - 1);   // this row's first lane in the warp
-    const int64_t row = (int64_t)blockIdx.x * (kThreadsA / kLanes) + threadIdx.x / kLanes;
+    const int64_t row = cta * (kThreadsA / kLanes) + threadIdx.x / kLanes;
     const int ngroups = bw / 16;
     const bool active = row < rows;
     const bool has0 = 2 * lane < ngroups, has1 = 2 * lane + 1 < ngroups;
@@ -188,8 +193,8 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool va
 }
 
 __device__ __forceinline__ void gptq_load_chunk(float* Es, float* Ut, const float* __restrict__ Et, int64_t ldE,
-                                                const float* __restrict__ U, int64_t rows, int64_t cols, int64_t j0,
-                                                int bw, int kc, int64_t r0, int64_t c0)
+                                                const float* __restrict__ U, int64_t rows, int64_t cols, int64_t cend,
+                                                int64_t j0, int bw, int kc, int64_t r0, int64_t c0)
 {
     // 32 x 128 floats each, 16 bytes per copy: 4 copies of each per thread
 #pragma unroll
@@ -198,23 +203,24 @@ __device__ __forceinline__ void gptq_load_chunk(float* Es, float* Ut, const floa
         const int k = i / (kTB / 4), t = (i % (kTB / 4)) * 4;
         const bool kin = kc + k < bw;
         const bool ein = kin && r0 + t < rows;       // ldE is a multiple of 4: a 4-row group is all in or all out
-        const bool uin = kin && c0 + t < cols;       // cols is a multiple of 16
+        const bool uin = kin && c0 + t < cend;       // cend is a multiple of 16
         cp_async16(Es + k * kTB + t, ein ? Et + (int64_t)(kc + k) * ldE + r0 + t : Et, ein);
         cp_async16(Ut + k * kTB + t, uin ? U + (j0 + kc + k) * cols + c0 + t : U, uin);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-__global__ void __launch_bounds__(256, 2)
-gptq_update_kernel(float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0, int bw,
-                   const float* __restrict__ U, const float* __restrict__ Et, int64_t ldE)
+__device__ __forceinline__ void gptq_update_body(int64_t tile, int64_t row_tiles, float* sm, float* __restrict__ w,
+                                                 int64_t rows, int64_t cols, int64_t j0, int bw,
+                                                 int64_t cfrom, int64_t cto, const float* __restrict__ U,
+                                                 const float* __restrict__ Et, int64_t ldE)
 {
-    extern __shared__ __align__(16) float sm[];      // 2 x {E chunk [k][row], U chunk [k][column]}
-    const int64_t r0 = (int64_t)blockIdx.x * kTB;
-    const int64_t c0 = j0 + bw + (int64_t)blockIdx.y * kTB;
+    // sm: 2 x {E chunk [k][row], U chunk [k][column]}
+    const int64_t r0 = (tile % row_tiles) * kTB;
+    const int64_t c0 = cfrom + (tile / row_tiles) * kTB;   // the tile's columns stop at cto (a multiple of 16)
     const int tr = (threadIdx.x >> 4) * 4, tc = (threadIdx.x & 15) * 4;
     const int nchunks = (bw + kBK - 1) / kBK;
-    gptq_load_chunk(sm, sm + kBK * kTB, Et, ldE, U, rows, cols, j0, bw, 0, r0, c0);
+    gptq_load_chunk(sm, sm + kBK * kTB, Et, ldE, U, rows, cols, cto, j0, bw, 0, r0, c0);
     // the tile's current values, four columns per 16-byte load (cols is a
     // multiple of 16, so a group of four is all in or all out)
     float acc[8][8];
@@ -225,7 +231,7 @@ gptq_update_kernel(float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0
         for (int h = 0; h < 2; ++h) {
             const int64_t cc = c0 + tc + 64 * h;
             float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            if (r < rows && cc < cols) v = *reinterpret_cast<const float4*>(w + r * cols + cc);
+            if (r < rows && cc < cto) v = *reinterpret_cast<const float4*>(w + r * cols + cc);
             acc[i][4 * h + 0] = v.x; acc[i][4 * h + 1] = v.y; acc[i][4 * h + 2] = v.z; acc[i][4 * h + 3] = v.w;
         }
     }
@@ -234,7 +240,7 @@ gptq_update_kernel(float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0
         float* Ut = Es + kBK * kTB;
         if (ch + 1 < nchunks) {
             float* En = sm + ((ch + 1) & 1) * 2 * kBK * kTB;
-            gptq_load_chunk(En, En + kBK * kTB, Et, ldE, U, rows, cols, j0, bw, (ch + 1) * kBK, r0, c0);
+            gptq_load_chunk(En, En + kBK * kTB, Et, ldE, U, rows, cols, cto, j0, bw, (ch + 1) * kBK, r0, c0);
             asm volatile("cp.async.wait_group 1;" ::: "memory");
         } else {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -261,45 +267,99 @@ gptq_update_kernel(float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int64_t cc = c0 + tc + 64 * h;
-            if (r < rows && cc < cols)
+            if (r < rows && cc < cto)
                 *reinterpret_cast<float4*>(w + r * cols + cc) =
                     make_float4(acc[i][4 * h + 0], acc[i][4 * h + 1], acc[i][4 * h + 2], acc[i][4 * h + 3]);
         }
     }
 }
 
+// The trailing update of one block's errors on columns [cfrom, cto).
+__global__ void __launch_bounds__(256, 2)
+gptq_update_kernel(float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0, int bw, int64_t cfrom,
+                   int64_t cto, const float* __restrict__ U, const float* __restrict__ Et, int64_t ldE)
+{
+    extern __shared__ __align__(16) float sm[];
+    const int64_t row_tiles = (rows + kTB - 1) / kTB;
+    gptq_update_body(blockIdx.x, row_tiles, sm, w, rows, cols, j0, bw, cfrom, cto, U, Et, ldE);
+}
+
+// One step of the pipeline: thread blocks [0, nA) run the in-block GPTQ of the
+// block at j0 (errors to Et); the others apply the previous block's errors
+// (Ep, block jp of width bwp) to the columns from j0 + bw on.  The two halves
+// touch disjoint columns of w: the in-block half only the block at j0 (whose
+// update by the previous block the preceding launch already applied), the
+// update half only the columns after it.  The in-block thread blocks come
+// first so that they start first; the update tiles fill the rest of the GPU
+// around them.
+__global__ void __launch_bounds__(256, 2)
+gptq_step_kernel(float* __restrict__ w, int64_t rows, int64_t cols, int64_t j0, int bw, int64_t nA,
+                 const float* __restrict__ U, const float* __restrict__ d_amax, uint8_t* __restrict__ codes,
+                 uint8_t* __restrict__ scales, float* __restrict__ d_S, float* __restrict__ deq,
+                 float* __restrict__ Et, const float* __restrict__ Ep, int64_t jp, int bwp, int64_t ldE,
+                 int32_t* __restrict__ d_status, float neg_zero)
+{
+    extern __shared__ __align__(16) float smem[];
+    __shared__ NvTables tb;
+    if ((int64_t)blockIdx.x < nA) {
+        gptq_block_body(blockIdx.x, smem, tb, w, rows, cols, j0, bw, U, d_amax, codes, scales, d_S, deq, Et, ldE,
+                        d_status, neg_zero);
+    } else {
+        const int64_t row_tiles = (rows + kTB - 1) / kTB;
+        gptq_update_body((int64_t)blockIdx.x - nA, row_tiles, smem, w, rows, cols, jp, bwp, j0 + bw, cols, U, Ep,
+                         ldE);
+    }
+}
+
 }  // namespace
 
-// Workspace: the block's scaled errors, transposed ([128][ldE] with ldE the
-// row count rounded up to a multiple of 4, so every 16-byte copy is aligned).
+// Workspace: the scaled errors of two consecutive blocks, each transposed
+// ([128][ldE] with ldE the row count rounded up to a multiple of 4, so every
+// 16-byte copy is aligned): the in-block step of block J writes one buffer
+// while the trailing update of block J-1 still reads the other.
 static int64_t gptq_ld(int64_t rows) { return (rows + 3) / 4 * 4; }
 
-size_t gptq_workspace_bytes(int64_t rows) { return (size_t)gptq_ld(rows) * kB * sizeof(float); }
+size_t gptq_workspace_bytes(int64_t rows) { return (size_t)2 * gptq_ld(rows) * kB * sizeof(float); }
 
+// Blocks J = 0, 1, ... of 128 columns.  Step J is one launch: the in-block
+// GPTQ of block J beside the update of block J-1's errors on the columns
+// from block J+1 on; then a small launch applies block J's errors to block
+// J+1's columns, which step J+1 needs.  Every element receives the errors of
+// the blocks before it in ascending order (the update of J-1 on block J+1's
+// columns runs in step J, before the launch that applies J's), so the bytes
+// are those of the column-by-column definition.
 cudaError_t launch_nvfp4_gptq(float* w, int64_t rows, int64_t cols, const float* U, const float* d_amax,
                               uint8_t* codes, uint8_t* scales, float* d_S, float* deq, float* E, int32_t* d_status,
                               cudaStream_t s)
 {
-    const size_t smem_a_max = (size_t)kB * kB * sizeof(float);
-    const size_t smem_b = (size_t)4 * kBK * kTB * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(gptq_block_kernel),
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a_max);
+    const size_t smem = (size_t)4 * kBK * kTB * sizeof(float);     // = kB * kB floats, the in-block need
+    static_assert(4 * kBK * kTB == kB * kB, "the two halves of the step kernel share one dynamic allocation");
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(gptq_step_kernel),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(reinterpret_cast<const void*>(gptq_update_kernel),
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b);
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t ldE = gptq_ld(rows);
-    const unsigned grid_a = (unsigned)((rows + (kThreadsA / kLanes) - 1) / (kThreadsA / kLanes));
-    for (int64_t j0 = 0; j0 < cols; j0 += kB) {
+    float* Ebuf[2] = {E, E + kB * ldE};
+    const int64_t nA = (rows + (kThreadsA / kLanes) - 1) / (kThreadsA / kLanes);
+    const int64_t row_tiles = (rows + kTB - 1) / kTB;
+    int bwp = 0;
+    int parity = 0;
+    for (int64_t j0 = 0; j0 < cols; j0 += kB, parity ^= 1) {
         const int bw = (int)(cols - j0 < kB ? cols - j0 : kB);
-        const size_t smem_a = (size_t)bw * bw * sizeof(float);
-        gptq_block_kernel<<<grid_a, kThreadsA, smem_a, s>>>(w, rows, cols, j0, bw, U, d_amax, codes, scales, d_S,
-                                                            deq, E, ldE, d_status, -0.0f);
-        const int64_t rem = cols - j0 - bw;
-        if (rem > 0) {
-            const dim3 grid_b((unsigned)((rows + kTB - 1) / kTB), (unsigned)((rem + kTB - 1) / kTB));
-            gptq_update_kernel<<<grid_b, 256, smem_b, s>>>(w, rows, cols, j0, bw, U, E, ldE);
-        }
+        // step: in-block j0, and block j0 - 128's errors on the columns from j0 + bw on
+        const int64_t rem = j0 > 0 ? cols - j0 - bw : 0;
+        const int64_t nB = rem > 0 ? row_tiles * ((rem + kTB - 1) / kTB) : 0;
+        gptq_step_kernel<<<(unsigned)(nA + nB), kThreadsA, smem, s>>>(
+            w, rows, cols, j0, bw, nA, U, d_amax, codes, scales, d_S, deq, Ebuf[parity], Ebuf[parity ^ 1],
+            j0 - kB, bwp, ldE, d_status, -0.0f);
+        // this block's errors on the next block's columns
+        const int64_t c1 = j0 + bw, c2 = c1 + kB < cols ? c1 + kB : cols;
+        if (c2 > c1)
+            gptq_update_kernel<<<(unsigned)(row_tiles * ((c2 - c1 + kTB - 1) / kTB)), 256, smem, s>>>(
+                w, rows, cols, j0, bw, c1, c2, U, Ebuf[parity], ldE);
+        bwp = bw;
     }
     return cudaGetLastError();
 }

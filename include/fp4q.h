@@ -287,7 +287,9 @@ fp4q_status fp4q_mxfp4_unrotate(const void* y, fp4q_dtype dt, int64_t rows, int6
                                 const uint32_t* sign_masks, void* out, fp4q_stream_t stream);
 
 /*
- * fp4q_gptq_workspace_bytes -- workspace of fp4q_nvfp4_gptq: rows * 128 floats.
+ * fp4q_gptq_workspace_bytes -- workspace of fp4q_nvfp4_gptq: the scaled errors
+ * of two consecutive 128-column blocks, 2 * 128 * ceil4(rows) floats
+ * (ceil4: rounded up to a multiple of 4); 0 for rows <= 0.
  */
 size_t fp4q_gptq_workspace_bytes(int64_t rows);
 
@@ -314,7 +316,10 @@ size_t fp4q_gptq_workspace_bytes(int64_t rows);
  *   codes, scales_e4m3, d_global_scale, deq (fp32, may be NULL) as
  *              fp4q_nvfp4_sweepmse.
  *   workspace  device, 16-byte aligned, fp4q_gptq_workspace_bytes(rows).
- * 2 * ceil(cols/128) launches.  Errors as fp4q_nvfp4_sweepmse, plus
+ * 2 * ceil(cols/128) - 1 launches: per block of 128 columns one launch runs
+ * the block's in-block GPTQ beside the trailing update of the previous
+ * block's errors, and a small one applies the block's errors to the next
+ * block.  Errors as fp4q_nvfp4_sweepmse, plus
  * FP4Q_ERR_ARG for a small workspace and FP4Q_ERR_SHAPE for cols > 2^20.
  */
 fp4q_status fp4q_nvfp4_gptq(float* w, int64_t rows, int64_t cols, const float* U, const float* d_amax,

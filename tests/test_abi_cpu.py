@@ -161,7 +161,7 @@ def test_widening_entries_argument_errors_without_a_gpu(fq):
     assert lib.fp4q_mxfp4_unrotate(None, 1, 0, 32, None, None, None) == fq.OK
     # GPTQ: shape, pointers, workspace size
     ws = fq.fp4q_gptq_workspace_bytes(4)
-    assert ws == 4 * 128 * 4 and fq.fp4q_gptq_workspace_bytes(0) == 0
+    assert ws == 2 * 4 * 128 * 4 and fq.fp4q_gptq_workspace_bytes(0) == 0
     assert lib.fp4q_nvfp4_gptq(q, 4, 24, q, q, q, q, q, None, q, ws, q, None) == fq.ERR_SHAPE
     assert lib.fp4q_nvfp4_gptq(q, 4, 16, None, q, q, q, q, None, q, ws, q, None) == fq.ERR_NULL
     assert lib.fp4q_nvfp4_gptq(q, 4, 16, q, q, q, q, q, None, None, ws, q, None) == fq.ERR_NULL

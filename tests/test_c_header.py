@@ -45,7 +45,7 @@ int main(void)
     EXPECT(fp4q_probe_copy(p, buf + 1024, 24, NULL), FP4Q_ERR_SHAPE);
     EXPECT(fp4q_probe_copy(buf + 8, buf + 1024, 32, NULL), FP4Q_ERR_ALIGN);
     if (fp4q_mma_scale_bytes(130, 6) != 2 * 2 * 512) { printf("FAIL mma bytes\n"); ++fails; }
-    if (fp4q_gptq_workspace_bytes(5) != 8 * 128 * 4) { printf("FAIL gptq workspace\n"); ++fails; }
+    if (fp4q_gptq_workspace_bytes(5) != 2 * 8 * 128 * 4) { printf("FAIL gptq workspace\n"); ++fails; }
     printf(fails ? "failed\n" : "ok\n");
     return fails != 0;
 }
