@@ -498,11 +498,11 @@ def run_reference(args):
 # so a launch of n elements moves about n times the per-element figure.  Once
 # the sources differ the figures no longer describe the kernel and none is
 # reported.
-NVFP4_PROFILE = {"bytes_per_element": (268480768 + 286225664) / (16384 * 8192),
-                 "warp_inst_per_element": 225.4e6 / (16384 * 8192),
-                 "issue_active_pct": 79.2,
+NVFP4_PROFILE = {"bytes_per_element": (268508928 + 287904768) / (16384 * 8192),
+                 "warp_inst_per_element": 215608887 / (16384 * 8192),
+                 "issue_active_pct": 77.96,
                  "sources": ("nvfp4.cu", "nvfp4_block.cuh", "screen.cuh", "device.cuh"),
-                 "sha256": "eeaccfe992e1af1b0984c8a9ffe3cbcc1d13d088c6b8c2383109abd62a785fc2"}
+                 "sha256": "3e86cf6431b7185a316bec64b57d7e3194bb7af91f2ca4a0a130342d81aaf892"}
 
 
 def nvfp4_profile_current():
