@@ -529,7 +529,7 @@ SINGLE_PATHS = {
     "nvfp4-wmse": (B_NVFP4, "nvfp4_sweep_kernel WMSE"),
     "mxfp4": (B_MXFP4, "mxfp4_kernel"),
     "mxfp4-absmax": (B_MXFP4, "mxfp4_kernel with the fused global max"),
-    "mxfp4-hadamard": (B_MXFP4, "mxfp4_kernel Hadamard"),
+    "mxfp4-hadamard": (B_MXFP4, "mxfp4_rot_pf_kernel (Hadamard, next block loaded during the current one)"),
     "dequant-nvfp4": (0.5 + 1.0 / 16 + 2.0, "dequant_kernel NVFP4"),
     "mma-layout": (2.0 / 16, "mma_scale_layout_kernel (NVFP4 scales, read + write)"),
     "focus-nvfp4": (2.0 + 1.0 / 16 + 2.0 / 8 + 0.5 + 2.0, "focus_kernel NVFP4, sub-blocks of 8"),

@@ -20,12 +20,17 @@ int resident_blocks_per_sm(const void* kernel, int threads, size_t dyn_smem);
 // two generations of resident thread blocks (a thread block that finishes early
 // is replaced, which evens out the tail), never more blocks than the work needs.
 template <typename Kernel>
-inline int64_t resident_grid(Kernel kernel, int threads, size_t dyn_smem, int64_t work_items)
+inline int64_t grid_rounds(Kernel kernel, int threads, size_t dyn_smem, int64_t work_items)
 {
     const int per_sm = resident_blocks_per_sm(reinterpret_cast<const void*>(kernel), threads, dyn_smem);
     const int64_t per_gen = (int64_t)per_sm * sm_count() * threads * 2;
     const int64_t rounds = (work_items + per_gen - 1) / per_gen;
-    const int64_t share = rounds < 1 ? 1 : rounds;
+    return rounds < 1 ? 1 : rounds;
+}
+template <typename Kernel>
+inline int64_t resident_grid(Kernel kernel, int threads, size_t dyn_smem, int64_t work_items)
+{
+    const int64_t share = grid_rounds(kernel, threads, dyn_smem, work_items);
     const int64_t g = (work_items + threads * share - 1) / (threads * share);
     return g < 1 ? 1 : g;
 }

@@ -28,6 +28,32 @@ namespace fp4q {
 
 constexpr float kInvSqrt32 = 0x1.6a09e6p-3f;   // RN(1/sqrt(32))
 
+// The 32 bf16 elements of a block from its 64 raw bytes, and max|w| as bits.
+__device__ __forceinline__ void unpack32_bf16_amax(const uint4* u, float (&x)[32], uint32_t& wmax)
+{
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        const uint4 t = u[v];
+        bf16x2_to_f32(t.x, x[8 * v + 0], x[8 * v + 1]);
+        bf16x2_to_f32(t.y, x[8 * v + 2], x[8 * v + 3]);
+        bf16x2_to_f32(t.z, x[8 * v + 4], x[8 * v + 5]);
+        bf16x2_to_f32(t.w, x[8 * v + 6], x[8 * v + 7]);
+        m2 = __vmaxu2(m2, __vmaxu2(t.x & 0x7FFF7FFFu, t.y & 0x7FFF7FFFu));
+        m2 = __vmaxu2(m2, __vmaxu2(t.z & 0x7FFF7FFFu, t.w & 0x7FFF7FFFu));
+    }
+    wmax = max(m2 & 0xFFFFu, m2 >> 16) << 16;
+}
+
+// max(bits_of(m), |v|) as binary32 bits, m a non-negative float's bits: a NaN
+// input gives the canonical NaN 0x7FFFFFFF, above Inf, above every finite value.
+__device__ __forceinline__ uint32_t max_nan_abs(uint32_t m, float v)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(__uint_as_float(m)), "f"(fabsf(v)));
+    return __float_as_uint(r);
+}
+
 // Neighbour-paired form (elements 2j, 2j+1 in a register pair).
 template <typename T, bool HAD>
 __device__ __forceinline__ uint32_t mxfp4_block_pairs_of_neighbours(const T* __restrict__ src, uint32_t sign_mask,
@@ -175,11 +201,16 @@ __device__ __forceinline__ uint32_t mxfp4_block_pairs_of_neighbours(const T* __r
 }
 
 // Half-paired form (elements j, j+16 in a register pair), for the rotation.
-template <typename T, bool HAD>
+// PF < 0: the block is loaded from src here.  PF >= 0 (bf16 only): the block's
+// 64 bytes arrive in `cur`, and the 64 bytes at `next` (if not null) are loaded
+// into `nxt` before any of this block's work.
+template <typename T, bool HAD, int PF = -1>
 __device__ __forceinline__ uint32_t mxfp4_block_pairs_of_halves(const T* __restrict__ src, uint32_t sign_mask,
                                                 uint8_t* __restrict__ codes16, uint8_t* __restrict__ scale,
                                                 T* __restrict__ deq32, float* __restrict__ loss,
-                                                int32_t* __restrict__ d_status, uint64_t z2, float neg_zero)
+                                                int32_t* __restrict__ d_status, uint64_t z2, float neg_zero,
+                                                const uint4* cur = nullptr, const T* __restrict__ next = nullptr,
+                                                uint4* nxt = nullptr)
 {
     // The block lives in 16 register pairs P[j].  With the rotation, P[j]
     // holds elements j and j+16: the butterfly stages h = 1, 2, 4, 8 act on
@@ -191,7 +222,13 @@ __device__ __forceinline__ uint32_t mxfp4_block_pairs_of_halves(const T* __restr
 #define FP4Q_E(j, h) (HAD ? (j) + 16 * (h) : 2 * (j) + (h))
     float x[32];
     uint32_t wmax;         // max |w| bits of the unrotated block
-    load_block_amax<32>(src, x, wmax);
+    if constexpr (PF < 0) {
+        load_block_amax<32>(src, x, wmax);
+    } else {
+        unpack32_bf16_amax(cur, x, wmax);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) nxt[v] = next ? ld_stream(next + 8 * v) : make_uint4(0, 0, 0, 0);
+    }
     uint32_t abits = wmax; // max |y| bits of the block that is quantized
     uint64_t P[16];
     if (HAD) {
@@ -219,7 +256,7 @@ __device__ __forceinline__ uint32_t mxfp4_block_pairs_of_halves(const T* __restr
             upk(P[j], a, c);
             P[j] = mul2(pk(__fadd_rn(a, c), __fsub_rn(a, c)), c2);
             upk(P[j], a, c);
-            abits = max(abits, max(__float_as_uint(a) & 0x7FFFFFFFu, __float_as_uint(c) & 0x7FFFFFFFu));
+            abits = max_nan_abs(max_nan_abs(abits, a), c);
         }
     } else {
 #pragma unroll
