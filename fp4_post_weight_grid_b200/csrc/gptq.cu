@@ -50,6 +50,11 @@ constexpr int kLanes = 4;         // threads per row in the in-block kernel: two
 constexpr int kThreadsA = 256;    // 64 rows per thread block
 constexpr int kTB = 128;          // output tile of the update kernel (rows and columns)
 constexpr int kBK = 32;           // block columns per shared-memory chunk of the update kernel
+// U's diagonal block in shared memory: row j of 128 columns, with 4 floats of
+// padding after every 32 columns, so that the four threads of a row (each
+// reading its own 32 columns) hit different banks.
+constexpr int kUs = kB + 16;
+__device__ __forceinline__ int us_at(int j, int c) { return j * kUs + c + 4 * (c >> 5); }
 
 // fma(-e, u, x) for the 16 values of one group, u from shared memory
 __device__ __forceinline__ void gptq_update16(float (&x)[16], float e, const float* __restrict__ u)
@@ -89,7 +94,7 @@ __device__ __forceinline__ void gptq_block_body(int64_t cta, float* Us, NvTables
     const NvScale c = nvfp4_scale(gmax);
     if (cta == 0 && threadIdx.x == 0 && j0 == 0) *d_S = c.S;
     for (int i = threadIdx.x; i < bw * bw; i += kThreadsA)
-        Us[i] = __ldg(U + (j0 + i / bw) * cols + j0 + i % bw);
+        Us[us_at(i / bw, i % bw)] = __ldg(U + (j0 + i / bw) * cols + j0 + i % bw);
     nvfp4_tables(tb, c.S);                           // synchronises: U's block is in place too
 
     const int lane = threadIdx.x & (kLanes - 1);
@@ -147,7 +152,7 @@ __device__ __forceinline__ void gptq_block_body(int64_t cta, float* Us, NvTables
                 float q, unused;
                 f16x2_to_f32(e2m1x2_to_f16x2(code), q, unused);
                 const float y = __fmul_rn(q, d);
-                e = __fdiv_rn(__fsub_rn(wj, y), Us[j * bw + j]);
+                e = __fdiv_rn(__fsub_rn(wj, y), Us[us_at(j, j)]);
                 nib |= (uint64_t)code << (4 * jj);
                 y4[jj & 3] = y;
                 if (active) {
@@ -157,7 +162,7 @@ __device__ __forceinline__ void gptq_block_body(int64_t cta, float* Us, NvTables
                 }
             }
             e = __shfl_sync(0xFFFFFFFFu, e, src0 + p);
-            const float* uj = Us + j * bw + 32 * lane;
+            const float* uj = Us + us_at(j, 32 * lane);
             if (lane > p) {
                 if (has0) gptq_update16(x0, e, uj);
                 if (has1) gptq_update16(x1, e, uj + 16);
@@ -332,8 +337,8 @@ cudaError_t launch_nvfp4_gptq(float* w, int64_t rows, int64_t cols, const float*
                               uint8_t* codes, uint8_t* scales, float* d_S, float* deq, float* E, int32_t* d_status,
                               cudaStream_t s)
 {
-    const size_t smem = (size_t)4 * kBK * kTB * sizeof(float);     // = kB * kB floats, the in-block need
-    static_assert(4 * kBK * kTB == kB * kB, "the two halves of the step kernel share one dynamic allocation");
+    // the two halves of the step kernel share one dynamic allocation
+    const size_t smem = (size_t)(kB * kUs > 4 * kBK * kTB ? kB * kUs : 4 * kBK * kTB) * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(gptq_step_kernel),
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
