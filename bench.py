@@ -215,6 +215,36 @@ class Model:
             self.chunks.append((items, ws, n, ev))
         self.launches_per_step = len(self.chunks)
 
+    def group_setup(self, size):
+        """Descriptors for the grouped calls: consecutive weights in groups of `size`
+        (7 = one layer), one MXFP4 and one NVFP4 launch per group."""
+        self.groups = []
+        for base in range(0, len(self.w), size):
+            idx = range(base, min(base + size, len(self.w)))
+            mx = [dict(w=self.w[i], amax=self.out[i]["amax"], mx_codes=self.out[i]["mx_codes"],
+                       mx_scales=self.out[i]["mx_scales"], mx_deq=self.out[i]["mx_deq"]) for i in idx]
+            nv = [dict(w=self.w[i], amax=self.out[i]["amax"], global_scale=self.out[i]["S"],
+                       nv_codes=self.out[i]["nv_codes"], nv_scales=self.out[i]["nv_scales"],
+                       nv_deq=self.out[i]["nv_deq"]) for i in idx]
+            ev = (torch.cuda.Event(enable_timing=True, external=True),
+                  torch.cuda.Event(enable_timing=True, external=True))
+            self.groups.append((mx, nv, torch.cuda.Event(), ev))
+        self.launches_per_step = 2 * len(self.groups)
+
+    def step_groups(self, stream, stream2):
+        """Per group: one MXFP4 launch (with each weight's max) on `stream`, then one
+        NVFP4 launch on `stream2` after it, overlapping the next group's MXFP4 launch."""
+        fq = self.fq
+        stream2.wait_stream(stream)
+        for mx, nv, ready, ev in self.groups:
+            fq.fp4q_mxfp4_quant_group(mx, self.status, stream)
+            ready.record(stream)
+            stream2.wait_event(ready)
+            ev[0].record(stream2)
+            fq.fp4q_nvfp4_sweep_group(nv, self.status, stream2)
+            ev[1].record(stream2)
+        stream.wait_stream(stream2)
+
     def step_batch(self, stream):
         """The whole model in one persistent launch per chunk of weights."""
         for items, ws, _, ev in self.chunks:
@@ -960,9 +990,11 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--streams", type=int, default=2, choices=[1, 2, 3, 4],
                     help="1: one stream; n > 1: MXFP4 passes on one stream, NVFP4 sweeps "
                          "round-robin on n - 1 more, each after its own tensor's MXFP4 pass")
-    ap.add_argument("--mode", default="calls", choices=["batch", "calls"],
+    ap.add_argument("--mode", default="calls", choices=["batch", "calls", "groups"],
                     help="batch: fp4q_quantize_batch (one persistent launch per chunk of weights); "
-                         "calls: two launches per weight (fp4q_mxfp4_quant_absmax + the NVFP4 sweep)")
+                         "calls: two launches per weight (fp4q_mxfp4_quant_absmax + the NVFP4 sweep); "
+                         "groups: fp4q_mxfp4_quant_group + fp4q_nvfp4_sweep_group per --group weights")
+    ap.add_argument("--group", type=int, default=7, help="weights per grouped launch (at most 32)")
     ap.add_argument("--chunk", type=int, default=128, help="weights per batch launch (at most 128)")
     ap.add_argument("--lag", type=int, default=0,
                     help="with --streams > 1: the MXFP4 pass of tensor t waits for the sweep of t - lag")
@@ -1009,10 +1041,14 @@ def main():
 
     if args.mode == "batch":
         model.batch_setup(args.chunk)
+    if args.mode == "groups":
+        model.group_setup(args.group)
 
     def run_step():
         if args.mode == "batch":
             model.step_batch(stream)
+        elif args.mode == "groups":
+            model.step_groups(stream, streams[1] if len(streams) > 1 else stream)
         elif args.streams == 1:
             model.step(stream)
         else:
@@ -1064,6 +1100,12 @@ def main():
         kern_ms = sum(ev[0].elapsed_time(ev[1]) for _, _, _, ev in model.chunks)
         kern_bytes = (B_NVFP4 + B_MXFP4) * n
         n_launch = len(model.chunks)
+    elif args.mode == "groups":
+        # the grouped NVFP4 sweep kernel: per-launch durations of the last timed step
+        kname = "nvfp4_group_kernel (MSE, bf16)"
+        kern_ms = sum(ev[0].elapsed_time(ev[1]) for _, _, _, ev in model.groups)
+        kern_bytes = B_NVFP4 * n
+        n_launch = len(model.groups)
     else:
         # the NVFP4 sweep kernel: per-launch durations of the last timed step
         kname = "nvfp4_sweep_kernel (MSE, bf16)"

@@ -32,7 +32,7 @@ __all__ = [
     "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout", "mma_scales",
     "fp4q_focus_quant", "fp4q_mxfp4_unrotate", "focus_quantize", "mxfp4_unrotate", "FocusResult",
     "fp4q_nvfp4_gptq", "fp4q_gptq_workspace_bytes", "nvfp4_gptq", "fp4q_probe_wait", "fp4q_probe_copy",
-    "quantize_batch",
+    "quantize_batch", "fp4q_mxfp4_quant_group", "fp4q_nvfp4_sweep_group", "GROUP_MAX",
     "NVFP4Result", "MXFP4Result", "nvfp4_quantize", "mxfp4_quantize", "quantize_dual", "dequantize",
     "FLAG_NONFINITE", "FLAG_RANGE", "FLAG_TIMEOUT",
 ]
@@ -47,6 +47,7 @@ F32, BF16 = 0, 1
 NVFP4, MXFP4 = 0, 1
 FLAG_NONFINITE, FLAG_RANGE, FLAG_TIMEOUT = 1, 2, 4
 BATCH_MAX = 128
+GROUP_MAX = 32
 NVFP4_BLOCK, MXFP4_BLOCK = 16, 32
 EXPORTS = ("fp4q_version", "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_global_absmax",
            "fp4q_nvfp4_sweepmse", "fp4q_nvfp4_sweepwmse", "fp4q_mxfp4_quant",
@@ -55,7 +56,7 @@ EXPORTS = ("fp4q_version", "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_g
            "fp4q_probe_e2m1", "fp4q_probe_e4m3", "fp4q_nvfp4_sweep_dynamic", "fp4q_dynamic_workspace_bytes",
            "fp4q_mma_scale_bytes", "fp4q_scales_to_mma_layout", "fp4q_focus_quant", "fp4q_mxfp4_unrotate",
            "fp4q_nvfp4_gptq", "fp4q_gptq_workspace_bytes", "fp4q_probe_wait",
-           "fp4q_probe_copy")
+           "fp4q_probe_copy", "fp4q_mxfp4_quant_group", "fp4q_nvfp4_sweep_group")
 
 
 class BatchTensor(ctypes.Structure):
@@ -121,6 +122,8 @@ def _load_locked():
     }
     sigs["fp4q_quantize_batch"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, ctypes.c_size_t, P, P]
     sigs["fp4q_quantize_batch_static"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, P]
+    sigs["fp4q_mxfp4_quant_group"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, P]
+    sigs["fp4q_nvfp4_sweep_group"] = [ctypes.POINTER(BatchTensor), ctypes.c_int32, I, P, P]
     sigs["fp4q_scales_to_mma_layout"] = [P, I64, I64, P, P]
     sigs["fp4q_focus_quant"] = [I, P, I, I64, I64, P, P, P, ctypes.c_int32, P, P, P, P, P]
     sigs["fp4q_mxfp4_unrotate"] = [P, I, I64, I64, P, P, P]
@@ -468,6 +471,60 @@ def fp4q_quantize_batch(items, workspace: torch.Tensor, d_status: torch.Tensor, 
     sp = _dev(d_status, "d_status", torch.int32, 1, dev)
     _check(load().fp4q_quantize_batch(arr, len(items), dt, wp, workspace.numel(), sp, _stream(stream)),
            "fp4q_quantize_batch")
+
+
+def _group_array(items, prefix):
+    """fp4q_batch_tensor array for a grouped call: w, amax and the `prefix`
+    ("mx" or "nv") outputs, plus sign_masks (mx) or importance and
+    global_scale (nv); the other fields stay NULL (argument marshalling)."""
+    dev = items[0]["w"].device
+    arr = (BatchTensor * len(items))()
+    for k, it in enumerate(items):
+        w = it["w"]
+        if w.dtype != items[0]["w"].dtype:
+            raise TypeError("all weights of a group share one dtype")
+        rows, cols = _rc(w, MXFP4_BLOCK if prefix == "mx" else NVFP4_BLOCK)
+        n = rows * cols
+        bs = MXFP4_BLOCK if prefix == "mx" else NVFP4_BLOCK
+        arr[k].w = _dev(w, "w", device=dev)
+        arr[k].rows, arr[k].cols = rows, cols
+        arr[k].amax = _dev(it["amax"], "amax", torch.float32, 1, dev)
+        if prefix == "mx":
+            arr[k].sign_masks = _dev(it.get("sign_masks"), "sign_masks", (torch.int32, torch.uint32),
+                                     cols // MXFP4_BLOCK, dev)
+        else:
+            arr[k].importance = _dev(it.get("importance"), "importance", torch.float32, cols, dev)
+            arr[k].global_scale = _dev(it["global_scale"], "global_scale", torch.float32, 1, dev)
+        setattr(arr[k], prefix + "_codes", _dev(it[prefix + "_codes"], prefix + "_codes", torch.uint8, n // 2, dev))
+        setattr(arr[k], prefix + "_scales", _dev(it[prefix + "_scales"], prefix + "_scales", torch.uint8, n // bs, dev))
+        setattr(arr[k], prefix + "_deq", _dev(it.get(prefix + "_deq"), prefix + "_deq", w.dtype, n, dev))
+        setattr(arr[k], prefix + "_loss", _dev(it.get(prefix + "_loss"), prefix + "_loss", torch.float32, n // bs, dev))
+    return arr, dev
+
+
+def fp4q_mxfp4_quant_group(items, d_status: torch.Tensor, stream=None) -> None:
+    """fp4q_mxfp4_quant_absmax for a list of weights in one launch per GROUP_MAX
+    weights of one kind.  `items`: dicts with w, amax, mx_codes, mx_scales
+    (CUDA tensors) and optionally sign_masks, mx_deq, mx_loss."""
+    if not items:
+        return
+    arr, dev = _group_array(items, "mx")
+    sp = _dev(d_status, "d_status", torch.int32, 1, dev)
+    _check(load().fp4q_mxfp4_quant_group(arr, len(items), _wdtype(items[0]["w"]), sp, _stream(stream)),
+           "fp4q_mxfp4_quant_group")
+
+
+def fp4q_nvfp4_sweep_group(items, d_status: torch.Tensor, stream=None) -> None:
+    """fp4q_nvfp4_sweepmse / fp4q_nvfp4_sweepwmse for a list of weights in one
+    launch per GROUP_MAX weights of one kind.  `items`: dicts with w, amax (the
+    weight's max|w|, already on the device), global_scale, nv_codes, nv_scales
+    (CUDA tensors) and optionally importance, nv_deq, nv_loss."""
+    if not items:
+        return
+    arr, dev = _group_array(items, "nv")
+    sp = _dev(d_status, "d_status", torch.int32, 1, dev)
+    _check(load().fp4q_nvfp4_sweep_group(arr, len(items), _wdtype(items[0]["w"]), sp, _stream(stream)),
+           "fp4q_nvfp4_sweep_group")
 
 
 def fp4q_dequant(fmt: int, codes, scales, d_global_scale, rows: int, cols: int, out,

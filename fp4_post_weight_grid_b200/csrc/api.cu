@@ -99,6 +99,55 @@ fp4q_status check_quant_args(const void* w, fp4q_dtype dt, int64_t rows, int64_t
     return FP4Q_OK;
 }
 
+// A grouped call: every descriptor is checked before anything is enqueued;
+// then the weights of each kind (kind(t): WMSE, or rotated) go out in
+// launches of at most kGroupMax, in list order.  fill() sets a launch item's
+// format-specific outputs.
+template <typename Check, typename Kind, typename Fill, typename Launch>
+fp4q_status group_call(const fp4q_batch_tensor* tensors, int32_t n, fp4q_dtype dt, int32_t* d_status,
+                              Check check, Kind kind, Fill fill, Launch launch)
+{
+    if (!valid_dtype(dt)) return FP4Q_ERR_DTYPE;
+    if (n < 0) return FP4Q_ERR_SHAPE;
+    if (n == 0) return FP4Q_OK;
+    if (!tensors || !d_status) return FP4Q_ERR_NULL;
+    if (!aligned(d_status, 4)) return FP4Q_ERR_ALIGN;
+    for (int32_t i = 0; i < n; ++i) {
+        const fp4q_status st = check(tensors[i]);
+        if (st != FP4Q_OK) return st;
+    }
+    for (int k = 0; k < 2; ++k) {
+        fp4q::GroupItem items[fp4q::kGroupMax];
+        int m = 0;
+        for (int32_t i = 0; i < n; ++i) {
+            const fp4q_batch_tensor& t = tensors[i];
+            if (kind(t) != (k == 1)) continue;
+            fp4q::GroupItem& it = items[m++];
+            it = fp4q::GroupItem{};
+            it.w = t.w;
+            it.rows = t.rows;
+            it.cols = t.cols;
+            it.importance = t.importance;
+            it.sign_masks = t.sign_masks;
+            it.amax = t.amax;
+            it.global_scale = t.global_scale;
+            fill(it, t);
+            if (m == fp4q::kGroupMax) {
+                launch(items, m, k == 1);
+                const fp4q_status st = after_launch();
+                if (st != FP4Q_OK) return st;
+                m = 0;
+            }
+        }
+        if (m > 0) {
+            launch(items, m, k == 1);
+            const fp4q_status st = after_launch();
+            if (st != FP4Q_OK) return st;
+        }
+    }
+    return FP4Q_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -435,6 +484,61 @@ fp4q_status fp4q_quantize_batch_static(const fp4q_batch_tensor* tensors, int32_t
         return FP4Q_ERR_CUDA;
     }
     return fp4q_quantize_batch(tensors, n, dt, ws, bytes, d_status, stream);
+}
+
+fp4q_status fp4q_mxfp4_quant_group(const fp4q_batch_tensor* tensors, int32_t n, fp4q_dtype dt,
+                                   int32_t* d_status, fp4q_stream_t stream)
+{
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    auto check = [&](const fp4q_batch_tensor& t) {
+        if (!shape_ok(t.rows, t.cols, FP4Q_MXFP4_BLOCK)) return FP4Q_ERR_SHAPE;
+        if (!t.amax) return FP4Q_ERR_NULL;
+        if (!aligned(t.amax, 4)) return FP4Q_ERR_ALIGN;
+        bool empty = false;
+        const fp4q_status st = check_quant_args(t.w, dt, t.rows, t.cols, FP4Q_MXFP4_BLOCK, t.mx_codes, t.mx_scales,
+                                                d_status, t.mx_deq, t.mx_loss, 16, &empty);
+        if (st != FP4Q_OK) return st;
+        if (!empty && t.sign_masks && !aligned(t.sign_masks, 4)) return FP4Q_ERR_ALIGN;
+        return FP4Q_OK;
+    };
+    auto kind = [](const fp4q_batch_tensor& t) { return t.sign_masks != nullptr; };
+    auto fill = [](fp4q::GroupItem& it, const fp4q_batch_tensor& t) {
+        it.codes = t.mx_codes;
+        it.scales = t.mx_scales;
+        it.deq = t.mx_deq;
+        it.loss = t.mx_loss;
+    };
+    auto launch = [&](const fp4q::GroupItem* items, int m, bool had) {
+        fp4q::launch_mxfp4_group(items, m, dt == FP4Q_BF16, had, d_status, s);
+    };
+    return group_call(tensors, n, dt, d_status, check, kind, fill, launch);
+}
+
+fp4q_status fp4q_nvfp4_sweep_group(const fp4q_batch_tensor* tensors, int32_t n, fp4q_dtype dt,
+                                   int32_t* d_status, fp4q_stream_t stream)
+{
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    auto check = [&](const fp4q_batch_tensor& t) {
+        bool empty = false;
+        const fp4q_status st = check_quant_args(t.w, dt, t.rows, t.cols, FP4Q_NVFP4_BLOCK, t.nv_codes, t.nv_scales,
+                                                d_status, t.nv_deq, t.nv_loss, 8, &empty);
+        if (st != FP4Q_OK || empty) return st;
+        if (!t.amax || !t.global_scale) return FP4Q_ERR_NULL;
+        if (!aligned(t.amax, 4) || !aligned(t.global_scale, 4) || (t.importance && !aligned(t.importance, 16)))
+            return FP4Q_ERR_ALIGN;
+        return FP4Q_OK;
+    };
+    auto kind = [](const fp4q_batch_tensor& t) { return t.importance != nullptr; };
+    auto fill = [](fp4q::GroupItem& it, const fp4q_batch_tensor& t) {
+        it.codes = t.nv_codes;
+        it.scales = t.nv_scales;
+        it.deq = t.nv_deq;
+        it.loss = t.nv_loss;
+    };
+    auto launch = [&](const fp4q::GroupItem* items, int m, bool wmse) {
+        fp4q::launch_nvfp4_group(items, m, dt == FP4Q_BF16, wmse, d_status, s);
+    };
+    return group_call(tensors, n, dt, d_status, check, kind, fill, launch);
 }
 
 fp4q_status fp4q_dequant(fp4q_format format, const uint8_t* codes, const uint8_t* scales,

@@ -5,6 +5,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "fp4q.h"
+
 namespace fp4q {
 
 // Number of SMs of the current device (cached per device).
@@ -38,6 +40,27 @@ inline int64_t resident_grid(Kernel kernel, int threads, size_t dyn_smem, int64_
 // Global max|x| into *d_amax; with d_status != nullptr a one-warp kernel then
 // flags a non-finite or out-of-range result.
 void launch_absmax(const void* x, bool bf16, int64_t n, float* d_amax, int32_t* d_status, cudaStream_t s);
+
+// One weight of a grouped launch (the fields the format's kernel reads;
+// importance selects WMSE for NVFP4, sign_masks the rotation for MXFP4).
+struct GroupItem {
+    const void* w;
+    int64_t rows, cols;
+    const float* importance;
+    const uint32_t* sign_masks;
+    float* amax;                 // NVFP4: read; MXFP4: written (max|w|)
+    float* global_scale;         // NVFP4: written
+    uint8_t* codes;
+    uint8_t* scales;
+    void* deq;
+    float* loss;
+};
+constexpr int kGroupMax = FP4Q_GROUP_MAX;    // weights per grouped launch
+
+// Grouped launches over items[0..n), n <= kGroupMax, all of one dtype and one
+// kind (NVFP4: all MSE or all WMSE; MXFP4: all plain or all rotated).
+void launch_nvfp4_group(const GroupItem* items, int n, bool bf16, bool wmse, int32_t* d_status, cudaStream_t s);
+void launch_mxfp4_group(const GroupItem* items, int n, bool bf16, bool had, int32_t* d_status, cudaStream_t s);
 
 // NVFP4 ScaleSweep: importance == nullptr selects MSE (window -3..+7), otherwise
 // WMSE (window -8..+7).

@@ -1,5 +1,6 @@
-// mxfp4.cu -- MXFP4 kernel for one weight: one thread per 32-element block over
-// a grid-stride loop; the per-block work is mxfp4_block (mxfp4_block.cuh).
+// mxfp4.cu -- MXFP4 kernels for one weight and for a group of weights in one
+// launch: one thread per 32-element block over a grid-stride loop; the
+// per-block work is mxfp4_block (mxfp4_block.cuh).
 #include <type_traits>
 
 #include "device.cuh"
@@ -12,9 +13,6 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// AMAX: also reduce max|w| of the unrotated input into *gmax_bits (an atomic
-// max on the binary32 bit pattern, which keeps NaN and Inf), for the NVFP4
-// global scale of the same weight.
 template <typename T, bool HAD, bool AMAX>
 __global__ void __launch_bounds__(kThreads, 4)
 mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
@@ -43,6 +41,82 @@ mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
             if (threadIdx.x == 0 && wmax != 0u) atomicMax(gmax_bits, wmax);
         }
     }
+}
+
+// Several weights in one launch, each with the fused max: weight t owns
+// thread blocks [cta0, cta0 + nctas).
+struct MxGroupParams {
+    int32_t n;
+    struct Item {
+        const void* w;
+        const uint32_t* masks;
+        uint8_t* codes;
+        uint8_t* scales;
+        void* deq;
+        float* loss;
+        unsigned* gmax_bits;
+        int64_t nblocks, blocks_per_row, cta0, nctas;
+    } t[kGroupMax];
+};
+
+// The thread block's item sits in shared memory and its pointers are read
+// there on every block: kept in registers across the loop they would push the
+// 64-register kernel into spills.
+template <typename T, bool HAD>
+__global__ void __launch_bounds__(kThreads, 4)
+mxfp4_group_kernel(const __grid_constant__ MxGroupParams P, int32_t* __restrict__ d_status, float neg_zero)
+{
+    __shared__ MxGroupParams::Item it;
+    __shared__ uint32_t warp_max[kThreads / 32];
+    if (threadIdx.x == 0) {
+        int t = 0;
+        while (t + 1 < P.n && (int64_t)blockIdx.x >= P.t[t + 1].cta0) ++t;
+        it = P.t[t];
+    }
+    __syncthreads();
+    const uint64_t z2 = pk(neg_zero, neg_zero);
+    uint32_t wmax = 0;
+    const int64_t stride = it.nctas * kThreads;
+    for (int64_t b = ((int64_t)blockIdx.x - it.cta0) * kThreads + threadIdx.x; b < it.nblocks; b += stride) {
+        const uint32_t m = HAD ? __ldg(it.masks + (b % it.blocks_per_row)) : 0u;
+        T* deq = static_cast<T*>(it.deq);
+        const uint32_t bm = mxfp4_block<T, HAD>(static_cast<const T*>(it.w) + b * 32, m, it.codes + b * 16,
+                                                it.scales + b, deq ? deq + b * 32 : nullptr,
+                                                it.loss ? it.loss + b : nullptr, d_status, z2, neg_zero);
+        wmax = max(wmax, bm);
+    }
+    wmax = __reduce_max_sync(0xFFFFFFFFu, wmax);
+    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = wmax;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        wmax = threadIdx.x < kThreads / 32 ? warp_max[threadIdx.x] : 0u;
+        wmax = __reduce_max_sync(0xFFFFFFFFu, wmax);
+        if (threadIdx.x == 0 && wmax != 0u) atomicMax(it.gmax_bits, wmax);
+    }
+}
+
+template <typename T, bool HAD>
+void launch_group_typed(const GroupItem* items, int n, int32_t* d_status, cudaStream_t s)
+{
+    auto kernel = mxfp4_group_kernel<T, HAD>;
+    MxGroupParams P{};
+    int64_t total = 0;
+    for (int i = 0; i < n; ++i) total += items[i].rows * (items[i].cols / 32);
+    const int64_t rounds = grid_rounds(kernel, kThreads, 0, total);
+    int64_t cta = 0;
+    P.n = 0;
+    for (int i = 0; i < n; ++i) {
+        cudaMemsetAsync(items[i].amax, 0, sizeof(float), s);     // max over no elements: 0
+        const int64_t nblocks = items[i].rows * (items[i].cols / 32);
+        if (nblocks == 0) continue;
+        MxGroupParams::Item& d = P.t[P.n++];
+        d = {items[i].w, items[i].sign_masks, items[i].codes, items[i].scales, items[i].deq, items[i].loss,
+             reinterpret_cast<unsigned*>(items[i].amax), nblocks, items[i].cols / 32, cta,
+             (nblocks + kThreads * rounds - 1) / (kThreads * rounds)};
+        cta += d.nctas;
+    }
+    if (P.n == 0) return;
+    kernel<<<(unsigned)cta, kThreads, 0, s>>>(P, d_status, -0.0f);
 }
 
 // Rotated bf16 with at least two blocks per thread: the next block's 64 bytes
@@ -130,6 +204,17 @@ void launch_rot(const void* w, int64_t rows, int64_t cols, const uint32_t* masks
 }
 
 }  // namespace
+
+void launch_mxfp4_group(const GroupItem* items, int n, bool bf16, bool had, int32_t* d_status, cudaStream_t s)
+{
+    if (had) {
+        if (bf16) launch_group_typed<__nv_bfloat16, true>(items, n, d_status, s);
+        else launch_group_typed<float, true>(items, n, d_status, s);
+    } else {
+        if (bf16) launch_group_typed<__nv_bfloat16, false>(items, n, d_status, s);
+        else launch_group_typed<float, false>(items, n, d_status, s);
+    }
+}
 
 void launch_mxfp4(const void* w, bool bf16, int64_t rows, int64_t cols, const uint32_t* sign_masks,
                   uint8_t* codes, uint8_t* scales, void* deq, float* loss, int32_t* d_status,

@@ -487,6 +487,47 @@ fp4q_status fp4q_quantize_batch_static(const fp4q_batch_tensor* tensors, int32_t
                                        int32_t* d_status, fp4q_stream_t stream);
 
 /*
+ * fp4q_mxfp4_quant_group -- fp4q_mxfp4_quant_absmax for a list of weights,
+ * one launch per FP4Q_GROUP_MAX weights of one kind (plain and rotated
+ * weights go to separate launches, in list order).  The launch's thread
+ * blocks are split among its weights in proportion to their sizes, each block
+ * working on one weight exactly as the single call's kernel would, so a list
+ * of small weights does not leave the GPU idle at the end of each one.
+ * Results are identical to the single calls.
+ *   tensors   HOST array of n fp4q_batch_tensor descriptors (read during the
+ *             call only).  Read per weight: w, rows, cols (cols % 32 == 0),
+ *             sign_masks (NULL: plain MXFP4, else the block Hadamard masks),
+ *             amax (written: max|w| of the unrotated weight, 0 if empty),
+ *             mx_codes, mx_scales, mx_deq and mx_loss (deq/loss may be NULL);
+ *             the other fields are ignored.
+ *   dt, d_status, stream   as fp4q_mxfp4_quant_absmax.
+ * Errors as fp4q_mxfp4_quant_absmax; every descriptor is checked before
+ * anything is enqueued.
+ */
+#define FP4Q_GROUP_MAX 32
+
+fp4q_status fp4q_mxfp4_quant_group(const fp4q_batch_tensor* tensors, int32_t n, fp4q_dtype dt,
+                                   int32_t* d_status, fp4q_stream_t stream);
+
+/*
+ * fp4q_nvfp4_sweep_group -- fp4q_nvfp4_sweepmse / fp4q_nvfp4_sweepwmse for a
+ * list of weights, one launch per FP4Q_GROUP_MAX weights of one kind (MSE and
+ * WMSE weights go to separate launches), thread blocks split as in
+ * fp4q_mxfp4_quant_group (ScaleSweep summary, "Metodologia: ScaleSweep"
+ * secs. 2-3 per weight).  Results are identical to the single calls.
+ *   tensors   HOST array of n descriptors.  Read per weight: w, rows, cols
+ *             (cols % 16 == 0), importance (NULL: MSE window, else the WMSE
+ *             weights [cols]), amax (read: max|w|, e.g. written by
+ *             fp4q_mxfp4_quant_group earlier on the stream), global_scale
+ *             (written), nv_codes, nv_scales, nv_deq, nv_loss (deq/loss may be
+ *             NULL); the other fields are ignored.  An empty weight is skipped.
+ *   dt, d_status, stream   as fp4q_nvfp4_sweepmse.
+ * Errors as fp4q_nvfp4_sweepmse; every descriptor is checked first.
+ */
+fp4q_status fp4q_nvfp4_sweep_group(const fp4q_batch_tensor* tensors, int32_t n, fp4q_dtype dt,
+                                   int32_t* d_status, fp4q_stream_t stream);
+
+/*
  * fp4q_dequant -- decode codes and scales back to values.
  * NVFP4: out = RN(q * RN(E4M3(s) * S)), S = *d_global_scale; MXFP4:
  * out = q * 2^(b-127); then rounded to `out_dt`.  Reproduces the `deq` output

@@ -113,6 +113,54 @@ def test_batch_argument_errors_without_a_gpu(fq):
     assert lib.fp4q_quantize_batch(arr, 0, 1, None, 0, None, None) == fq.OK
 
 
+def test_group_argument_errors_without_a_gpu(fq):
+    lib = fq.load()
+    buf = ctypes.create_string_buffer(4096)
+    p = ctypes.addressof(buf)
+    p16 = p + (-p % 16)
+
+    def one(fn, **kw):
+        t = fq.BatchTensor()
+        for f, _ in fq.BatchTensor._fields_:
+            setattr(t, f, p16)
+        t.rows, t.cols, t.importance, t.sign_masks = 2, 64, None, None
+        t.nv_deq = t.nv_loss = t.mx_deq = t.mx_loss = None
+        for k, v in kw.items():
+            setattr(t, k, v)
+        arr = (fq.BatchTensor * 1)(t)
+        return getattr(lib, fn)(arr, 1, 1, p16, None)
+
+    for fn in ("fp4q_mxfp4_quant_group", "fp4q_nvfp4_sweep_group"):
+        assert one(fn, rows=-1) == fq.ERR_SHAPE
+        assert one(fn, w=None) == fq.ERR_NULL
+        assert one(fn, amax=None) == fq.ERR_NULL
+        assert one(fn, w=p16 + 2) == fq.ERR_ALIGN
+        assert one(fn, amax=p16 + 2) == fq.ERR_ALIGN
+        arr = (fq.BatchTensor * 1)()
+        assert getattr(lib, fn)(arr, 1, 9, p16, None) == fq.ERR_DTYPE
+        assert getattr(lib, fn)(arr, -1, 1, p16, None) == fq.ERR_SHAPE
+        assert getattr(lib, fn)(None, 1, 1, p16, None) == fq.ERR_NULL
+        assert getattr(lib, fn)(arr, 1, 1, None, None) == fq.ERR_NULL
+        assert getattr(lib, fn)(arr, 0, 1, None, None) == fq.OK
+    # per-format block sizes and outputs
+    assert one("fp4q_mxfp4_quant_group", cols=48) == fq.ERR_SHAPE
+    assert one("fp4q_nvfp4_sweep_group", cols=48) != fq.ERR_SHAPE          # 48 % 16 == 0: shape is fine
+    assert one("fp4q_mxfp4_quant_group", mx_codes=p16 + 8) == fq.ERR_ALIGN
+    assert one("fp4q_nvfp4_sweep_group", nv_codes=p16 + 4) == fq.ERR_ALIGN
+    assert one("fp4q_nvfp4_sweep_group", global_scale=None) == fq.ERR_NULL
+    assert one("fp4q_nvfp4_sweep_group", importance=p16 + 4) == fq.ERR_ALIGN
+    assert one("fp4q_mxfp4_quant_group", sign_masks=p16 + 2) == fq.ERR_ALIGN
+    # a later bad descriptor stops the call before anything is enqueued
+    good = fq.BatchTensor()
+    for f, _ in fq.BatchTensor._fields_:
+        setattr(good, f, p16)
+    good.rows, good.cols = 0, 64
+    bad = fq.BatchTensor()
+    bad.rows, bad.cols = 1, 40
+    arr = (fq.BatchTensor * 2)(good, bad)
+    assert lib.fp4q_mxfp4_quant_group(arr, 2, 1, p16, None) == fq.ERR_SHAPE
+
+
 def test_dynamic_argument_errors_without_a_gpu(fq):
     lib = fq.load()
     buf = ctypes.create_string_buffer(256)

@@ -44,6 +44,17 @@ int main(void)
     EXPECT(fp4q_mxfp4_unrotate(p, FP4Q_BF16, 1, 48, (const uint32_t*)buf, p, NULL), FP4Q_ERR_SHAPE);
     EXPECT(fp4q_probe_copy(p, buf + 1024, 24, NULL), FP4Q_ERR_SHAPE);
     EXPECT(fp4q_probe_copy(buf + 8, buf + 1024, 32, NULL), FP4Q_ERR_ALIGN);
+    {
+        fp4q_batch_tensor t;
+        memset(&t, 0, sizeof(t));
+        t.w = p; t.rows = 1; t.cols = 40;
+        EXPECT(fp4q_mxfp4_quant_group(&t, 1, FP4Q_BF16, st, NULL), FP4Q_ERR_SHAPE);
+        t.cols = 32;
+        EXPECT(fp4q_nvfp4_sweep_group(&t, 1, FP4Q_BF16, st, NULL), FP4Q_ERR_NULL);
+        EXPECT(fp4q_nvfp4_sweep_group(&t, -1, FP4Q_BF16, st, NULL), FP4Q_ERR_SHAPE);
+        EXPECT(fp4q_mxfp4_quant_group(&t, 0, FP4Q_BF16, NULL, NULL), FP4Q_OK);
+        if (FP4Q_GROUP_MAX < 8) { printf("FAIL group max\n"); ++fails; }
+    }
     if (fp4q_mma_scale_bytes(130, 6) != 2 * 2 * 512) { printf("FAIL mma bytes\n"); ++fails; }
     if (fp4q_gptq_workspace_bytes(5) != 2 * 8 * 128 * 4) { printf("FAIL gptq workspace\n"); ++fails; }
     printf(fails ? "failed\n" : "ok\n");
