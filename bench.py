@@ -215,12 +215,22 @@ class Model:
             self.chunks.append((items, ws, n, ev))
         self.launches_per_step = len(self.chunks)
 
-    def group_setup(self, size):
-        """Descriptors for the grouped calls: consecutive weights in groups of `size`
-        (7 = one layer), one MXFP4 and one NVFP4 launch per group."""
+    def group_setup(self, size, layer_sizes=None):
+        """Descriptors for the grouped calls, one MXFP4 and one NVFP4 launch per group:
+        consecutive weights in groups of `size` (7 = one layer), or each layer's seven
+        weights split into consecutive groups of `layer_sizes` (summing to 7)."""
         self.groups = []
-        for base in range(0, len(self.w), size):
-            idx = range(base, min(base + size, len(self.w)))
+        if layer_sizes:
+            per_layer = sum(layer_sizes)
+            bounds = []
+            for base in range(0, len(self.w), per_layer):
+                for k in layer_sizes:
+                    bounds.append((base, min(base + k, len(self.w))))
+                    base += k
+        else:
+            bounds = [(b, min(b + size, len(self.w))) for b in range(0, len(self.w), size)]
+        for lo, hi in bounds:
+            idx = range(lo, hi)
             mx = [dict(w=self.w[i], amax=self.out[i]["amax"], mx_codes=self.out[i]["mx_codes"],
                        mx_scales=self.out[i]["mx_scales"], mx_deq=self.out[i]["mx_deq"]) for i in idx]
             nv = [dict(w=self.w[i], amax=self.out[i]["amax"], global_scale=self.out[i]["S"],
@@ -229,20 +239,26 @@ class Model:
             ev = (torch.cuda.Event(enable_timing=True, external=True),
                   torch.cuda.Event(enable_timing=True, external=True))
             self.groups.append((mx, nv, torch.cuda.Event(), ev))
+        self.group_done = [torch.cuda.Event() for _ in self.groups]
         self.launches_per_step = 2 * len(self.groups)
 
-    def step_groups(self, stream, stream2):
+    def step_groups(self, stream, stream2, lag=0):
         """Per group: one MXFP4 launch (with each weight's max) on `stream`, then one
-        NVFP4 launch on `stream2` after it, overlapping the next group's MXFP4 launch."""
+        NVFP4 launch on `stream2` after it, overlapping the next group's MXFP4 launch;
+        with lag > 0 the MXFP4 launch of group g also waits for the NVFP4 launch of
+        group g - lag."""
         fq = self.fq
         stream2.wait_stream(stream)
-        for mx, nv, ready, ev in self.groups:
+        for g, (mx, nv, ready, ev) in enumerate(self.groups):
+            if lag > 0 and g >= lag:
+                stream.wait_event(self.group_done[g - lag])
             fq.fp4q_mxfp4_quant_group(mx, self.status, stream)
             ready.record(stream)
             stream2.wait_event(ready)
             ev[0].record(stream2)
             fq.fp4q_nvfp4_sweep_group(nv, self.status, stream2)
             ev[1].record(stream2)
+            self.group_done[g].record(stream2)
         stream.wait_stream(stream2)
 
     def step_batch(self, stream):
@@ -528,11 +544,12 @@ def run_reference(args):
 # so a launch of n elements moves about n times the per-element figure.  Once
 # the sources differ the figures no longer describe the kernel and none is
 # reported.
-NVFP4_PROFILE = {"bytes_per_element": (268508928 + 287904768) / (16384 * 8192),
-                 "warp_inst_per_element": 215608887 / (16384 * 8192),
-                 "issue_active_pct": 77.96,
+NVFP4_PROFILE = {"bytes_per_element": (268524544 + 287375616) / (16384 * 8192),
+                 "warp_inst_per_element": 220760623 / (16384 * 8192),
+                 "issue_active_pct": 78.18,
+                 "kernel": "nvfp4_group_kernel (MSE, bf16), one 16384x8192 weight",
                  "sources": ("nvfp4.cu", "nvfp4_block.cuh", "screen.cuh", "device.cuh"),
-                 "sha256": "3e86cf6431b7185a316bec64b57d7e3194bb7af91f2ca4a0a130342d81aaf892"}
+                 "sha256": "06fb432f7bd8acf96936c9b18bb88a2aadbe58d1ec144ea4acf4c55f63a514f7"}
 
 
 def nvfp4_profile_current():
@@ -560,6 +577,8 @@ SINGLE_PATHS = {
     "mxfp4": (B_MXFP4, "mxfp4_kernel"),
     "mxfp4-absmax": (B_MXFP4, "mxfp4_kernel with the fused global max"),
     "mxfp4-hadamard": (B_MXFP4, "mxfp4_rot_pf_kernel (Hadamard, next block loaded during the current one)"),
+    "nvfp4-mse-group": (B_NVFP4, "nvfp4_group_kernel MSE (fp4q_nvfp4_sweep_group, one weight)"),
+    "mxfp4-absmax-group": (B_MXFP4, "mxfp4_group_kernel (fp4q_mxfp4_quant_group, one weight)"),
     "dequant-nvfp4": (0.5 + 1.0 / 16 + 2.0, "dequant_kernel NVFP4"),
     "mma-layout": (2.0 / 16, "mma_scale_layout_kernel (NVFP4 scales, read + write)"),
     "focus-nvfp4": (2.0 + 1.0 / 16 + 2.0 / 8 + 0.5 + 2.0, "focus_kernel NVFP4, sub-blocks of 8"),
@@ -625,6 +644,12 @@ def run_single(args):
             fq.fp4q_probe_copy(w, deq, stream)
         elif args.single == "dequant-nvfp4":
             fq.fp4q_dequant(fq.NVFP4, codes, sc16, S, rows, cols, deq, stream)
+        elif args.single == "nvfp4-mse-group":
+            fq.fp4q_nvfp4_sweep_group([dict(w=w, amax=amax, global_scale=S, nv_codes=codes, nv_scales=sc16,
+                                            nv_deq=deq)], st, stream)
+        elif args.single == "mxfp4-absmax-group":
+            fq.fp4q_mxfp4_quant_group([dict(w=w, amax=amax, mx_codes=codes, mx_scales=sc32, mx_deq=deq)], st,
+                                      stream)
 
     times = []
     for i in range(args.warmup + args.steps):
@@ -990,14 +1015,17 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--streams", type=int, default=2, choices=[1, 2, 3, 4],
                     help="1: one stream; n > 1: MXFP4 passes on one stream, NVFP4 sweeps "
                          "round-robin on n - 1 more, each after its own tensor's MXFP4 pass")
-    ap.add_argument("--mode", default="calls", choices=["batch", "calls", "groups"],
+    ap.add_argument("--mode", default="groups", choices=["batch", "calls", "groups"],
                     help="batch: fp4q_quantize_batch (one persistent launch per chunk of weights); "
                          "calls: two launches per weight (fp4q_mxfp4_quant_absmax + the NVFP4 sweep); "
                          "groups: fp4q_mxfp4_quant_group + fp4q_nvfp4_sweep_group per --group weights")
-    ap.add_argument("--group", type=int, default=7, help="weights per grouped launch (at most 32)")
+    ap.add_argument("--group", type=int, default=4, help="weights per grouped launch (at most 32)")
+    ap.add_argument("--layer-groups", default="",
+                    help="split each layer's 7 weights (q,k,v,o,gate,up,down) into consecutive groups "
+                         "of these sizes, e.g. 3,2,1,1 (overrides --group)")
     ap.add_argument("--chunk", type=int, default=128, help="weights per batch launch (at most 128)")
     ap.add_argument("--lag", type=int, default=0,
-                    help="with --streams > 1: the MXFP4 pass of tensor t waits for the sweep of t - lag")
+                    help="with --streams > 1: the MXFP4 pass of tensor (or group) t waits for the sweep of t - lag")
     return ap
 
 
@@ -1042,13 +1070,14 @@ def main():
     if args.mode == "batch":
         model.batch_setup(args.chunk)
     if args.mode == "groups":
-        model.group_setup(args.group)
+        sizes = [int(v) for v in args.layer_groups.split(",")] if args.layer_groups else None
+        model.group_setup(args.group, sizes)
 
     def run_step():
         if args.mode == "batch":
             model.step_batch(stream)
         elif args.mode == "groups":
-            model.step_groups(stream, streams[1] if len(streams) > 1 else stream)
+            model.step_groups(stream, streams[1] if len(streams) > 1 else stream, args.lag)
         elif args.streams == 1:
             model.step(stream)
         else:
@@ -1127,7 +1156,8 @@ def main():
             explain.update({
                 "warp_instructions_per_element": ipe,
                 "issue_active_pct_of_active_cycles": prof["issue_active_pct"],
-                "basis": "ncu smsp__inst_executed.sum and smsp__issue_active on one 16384x8192 launch "
+                "basis": "ncu smsp__inst_executed.sum and smsp__issue_active on one 16384x8192 weight "
+                         "through the same kernel "
                          "(profiles/nvfp4_sweep_mse_16384x8192.md)",
                 "issue_bound_time_fraction": (n * ipe * 32 / issue_peak) / (kern_ms * 1e-3),
                 "issue_peak_lane_inst_per_s": issue_peak})

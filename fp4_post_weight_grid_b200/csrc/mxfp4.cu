@@ -60,29 +60,31 @@ struct MxGroupParams {
 };
 
 // The thread block's item sits in shared memory and its pointers are read
-// there on every block: kept in registers across the loop they would push the
-// 64-register kernel into spills.
+// there (volatile, so not hoisted into registers) at every block: held in
+// registers across the loop they push the 64-register kernel into spills.
 template <typename T, bool HAD>
 __global__ void __launch_bounds__(kThreads, 4)
 mxfp4_group_kernel(const __grid_constant__ MxGroupParams P, int32_t* __restrict__ d_status, float neg_zero)
 {
-    __shared__ MxGroupParams::Item it;
+    __shared__ MxGroupParams::Item item;
     __shared__ uint32_t warp_max[kThreads / 32];
     if (threadIdx.x == 0) {
         int t = 0;
         while (t + 1 < P.n && (int64_t)blockIdx.x >= P.t[t + 1].cta0) ++t;
-        it = P.t[t];
+        item = P.t[t];
     }
     __syncthreads();
+    const volatile MxGroupParams::Item& it = item;
     const uint64_t z2 = pk(neg_zero, neg_zero);
     uint32_t wmax = 0;
-    const int64_t stride = it.nctas * kThreads;
-    for (int64_t b = ((int64_t)blockIdx.x - it.cta0) * kThreads + threadIdx.x; b < it.nblocks; b += stride) {
+    for (int64_t b = ((int64_t)blockIdx.x - it.cta0) * kThreads + threadIdx.x; b < it.nblocks;
+         b += it.nctas * kThreads) {
         const uint32_t m = HAD ? __ldg(it.masks + (b % it.blocks_per_row)) : 0u;
         T* deq = static_cast<T*>(it.deq);
+        float* loss = it.loss;
         const uint32_t bm = mxfp4_block<T, HAD>(static_cast<const T*>(it.w) + b * 32, m, it.codes + b * 16,
                                                 it.scales + b, deq ? deq + b * 32 : nullptr,
-                                                it.loss ? it.loss + b : nullptr, d_status, z2, neg_zero);
+                                                loss ? loss + b : nullptr, d_status, z2, neg_zero);
         wmax = max(wmax, bm);
     }
     wmax = __reduce_max_sync(0xFFFFFFFFu, wmax);
