@@ -35,17 +35,33 @@ int resident_blocks_per_sm(const void* kernel, int threads, size_t dyn_smem)
 {
     static std::mutex mu;
     static std::map<std::tuple<const void*, int, int, size_t>, int> cache;   // (kernel, device, threads, smem)
+    static std::map<std::pair<const void*, int>, size_t> limit;              // (kernel, device) -> raised limit
     int dev = 0;
     cudaGetDevice(&dev);
     const auto key = std::make_tuple(kernel, dev, threads, dyn_smem);
     std::lock_guard<std::mutex> lock(mu);
+    // A kernel's dynamic shared memory limit is raised, never lowered: the
+    // default allows 48 KB, and setting a smaller limit for one size would make
+    // a later launch of the same kernel with more (a cached size) fail.
+    constexpr size_t kDefaultLimit = 48 * 1024;
+    if (dyn_smem > kDefaultLimit) {
+        size_t& cur = limit[std::make_pair(kernel, dev)];
+        if (dyn_smem > cur) {
+            if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem) ==
+                cudaSuccess)
+                cur = dyn_smem;
+            else
+                (void)cudaGetLastError();    // the launch reports it; keep it out of later status checks
+        }
+    }
     auto it = cache.find(key);
     if (it != cache.end()) return it->second;
-    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem);
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, dyn_smem) != cudaSuccess ||
-        per_sm <= 0)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, dyn_smem) != cudaSuccess) {
+        (void)cudaGetLastError();
         per_sm = 1;
+    }
+    if (per_sm <= 0) per_sm = 1;
     cache[key] = per_sm;
     return per_sm;
 }

@@ -14,8 +14,9 @@ int sm_count();
 
 // Resident thread blocks per SM of `kernel` with `threads` threads and
 // `dyn_smem` bytes of dynamic shared memory on the current device; raises the
-// kernel's dynamic shared memory limit the first time.  Cached per (kernel,
-// device, threads, dyn_smem).
+// kernel's dynamic shared memory limit to dyn_smem when that is above the
+// 48 KB default and above what was set before (never lowers it).  Cached per
+// (kernel, device, threads, dyn_smem).
 int resident_blocks_per_sm(const void* kernel, int threads, size_t dyn_smem);
 
 // Grid for a grid-stride kernel: the work is split into equal shares for about

@@ -131,13 +131,22 @@ void launch_group_typed(const GroupItem* items, int n, int32_t* d_status, cudaSt
 // gains 131 -> 125 us alone, but it runs beside the NVFP4 sweep in the
 // whole-model step, where its fewer resident warps cost more than they gain.)
 constexpr int kPfThreads = 256;
-template <bool AMAX>
+#ifndef FP4Q_SIGN_TABLE
+#define FP4Q_SIGN_TABLE 1
+#endif
+// TABLE: the sign flips come from a shared-memory table of every column
+// group's 16 sign words (bit 15 and bit 31 of the bf16 pair word k carry mask
+// bits 2k and 2k+1), built once per thread block and XORed into the raw words
+// before they are unpacked: four 16-byte shared loads and sixteen XORs per
+// block instead of a shift and a XOR per element.
+template <bool AMAX, bool TABLE>
 __global__ void __launch_bounds__(kPfThreads, 2)
 mxfp4_rot_pf_kernel(const __nv_bfloat16* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
                 const uint32_t* __restrict__ masks, uint8_t* __restrict__ codes,
                 uint8_t* __restrict__ scales, __nv_bfloat16* __restrict__ deq, float* __restrict__ loss,
                 int32_t* __restrict__ d_status, float neg_zero, unsigned* __restrict__ gmax_bits)
 {
+    extern __shared__ uint4 sign_tab[];               // TABLE: blocks_per_row x 4
     const uint64_t z2 = pk(neg_zero, neg_zero);
     uint32_t wmax = 0;
     const int64_t stride = (int64_t)gridDim.x * kPfThreads;
@@ -147,13 +156,36 @@ mxfp4_rot_pf_kernel(const __nv_bfloat16* __restrict__ w, int64_t nblocks, int64_
     uint4 u[4];
 #pragma unroll
     for (int v = 0; v < 4; ++v) u[v] = b < nblocks ? ld_stream(w + b * 32 + 8 * v) : make_uint4(0, 0, 0, 0);
+    if (TABLE) {
+        for (int64_t g = threadIdx.x; g < blocks_per_row; g += kPfThreads) {
+            const uint32_t m = __ldg(masks + g);
+            uint32_t sw[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) sw[k] = ((m >> (2 * k)) & 1u) << 15 | ((m >> (2 * k + 1)) & 1u) << 31;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) sign_tab[g * 4 + v] = make_uint4(sw[4 * v], sw[4 * v + 1], sw[4 * v + 2], sw[4 * v + 3]);
+        }
+        __syncthreads();
+    }
     for (; b < nblocks; b += stride) {
         const int64_t nb = b + stride;
         const __nv_bfloat16* next = nb < nblocks ? w + nb * 32 : nullptr;
         uint4 nu[4];
-        const uint32_t bm = mxfp4_block_pairs_of_halves<__nv_bfloat16, true, 0>(
-            nullptr, __ldg(masks + col), codes + b * 16, scales + b, deq ? deq + b * 32 : nullptr,
-            loss ? loss + b : nullptr, d_status, z2, neg_zero, u, next, nu);
+        uint32_t bm;
+        if (TABLE) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const uint4 t = sign_tab[col * 4 + v];
+                u[v] = make_uint4(u[v].x ^ t.x, u[v].y ^ t.y, u[v].z ^ t.z, u[v].w ^ t.w);
+            }
+            bm = mxfp4_block_pairs_of_halves<__nv_bfloat16, true, 0>(
+                nullptr, 0u, codes + b * 16, scales + b, deq ? deq + b * 32 : nullptr,
+                loss ? loss + b : nullptr, d_status, z2, neg_zero, u, next, nu);
+        } else {
+            bm = mxfp4_block_pairs_of_halves<__nv_bfloat16, true, 0>(
+                nullptr, __ldg(masks + col), codes + b * 16, scales + b, deq ? deq + b * 32 : nullptr,
+                loss ? loss + b : nullptr, d_status, z2, neg_zero, u, next, nu);
+        }
         col += step_col;
         if (col >= blocks_per_row) col -= blocks_per_row;
 #pragma unroll
@@ -180,9 +212,21 @@ void launch_typed(const void* w, int64_t rows, int64_t cols, const uint32_t* mas
 {
     const int64_t nblocks = rows * (cols / 32);
     if constexpr (HAD && std::is_same<T, __nv_bfloat16>::value) {
-        if (grid_rounds(mxfp4_rot_pf_kernel<AMAX>, kPfThreads, 0, nblocks) >= 2) {
-            const int64_t grid = resident_grid(mxfp4_rot_pf_kernel<AMAX>, kPfThreads, 0, nblocks);
-            mxfp4_rot_pf_kernel<AMAX><<<(unsigned)grid, kPfThreads, 0, s>>>(
+        const int64_t bpr = cols / 32;
+        if (FP4Q_SIGN_TABLE && bpr <= 1024) {            // table of at most 64 KB
+            auto kernel = mxfp4_rot_pf_kernel<AMAX, true>;
+            const size_t tab = (size_t)bpr * sizeof(uint4) * 4;
+            if (grid_rounds(kernel, kPfThreads, tab, nblocks) >= 2) {
+                const int64_t grid = resident_grid(kernel, kPfThreads, tab, nblocks);
+                kernel<<<(unsigned)grid, kPfThreads, tab, s>>>(
+                    static_cast<const __nv_bfloat16*>(w), nblocks, bpr, masks, codes, scales,
+                    static_cast<__nv_bfloat16*>(deq), loss, d_status, -0.0f, gmax_bits);
+                return;
+            }
+        }
+        if (grid_rounds(mxfp4_rot_pf_kernel<AMAX, false>, kPfThreads, 0, nblocks) >= 2) {
+            const int64_t grid = resident_grid(mxfp4_rot_pf_kernel<AMAX, false>, kPfThreads, 0, nblocks);
+            mxfp4_rot_pf_kernel<AMAX, false><<<(unsigned)grid, kPfThreads, 0, s>>>(
                 static_cast<const __nv_bfloat16*>(w), nblocks, cols / 32, masks, codes, scales,
                 static_cast<__nv_bfloat16*>(deq), loss, d_status, -0.0f, gmax_bits);
             return;

@@ -93,3 +93,30 @@ def test_prefetch_rotation_overflow_flag(weight):
     h = fq.mxfp4_quantize(w.to(DEV), torch.from_numpy(masks.view(np.int32)).to(DEV))
     torch.cuda.synchronize()
     assert int(h.status.item()) == fq.FLAG_NONFINITE
+
+
+def test_prefetch_rotated_wide_rows_without_the_sign_table():
+    """More than 1024 column groups (33,024 columns): the rotated kernel reads
+    each block's sign mask instead of a shared table of sign words; three
+    rounds with a ragged last one."""
+    rows, cols = 300, 33024
+    w = synth.t_weight(rows, cols, nu=4, scale=0.02, seed=63, device=DEV).cpu()
+    masks = synth.sign_masks(cols, seed=63)
+    sample = np.unique(np.concatenate([np.arange(0, rows, 23), [rows - 2, rows - 1]]))
+    mxfp4_parity(w, masks, rows_sample=sample)
+
+
+def test_rotated_calls_with_changing_table_sizes():
+    """The shared table of sign words grows with the column count (up to 64 KB,
+    above the 48 KB default limit).  Calls of different widths in any order
+    must all launch and stay bit-exact: a kernel's shared-memory limit is only
+    ever raised, so a narrow call cannot break a later wider one."""
+    for rows, cols in [(1200, 4096), (2400, 2048), (1200, 4096), (160, 32768), (2400, 2048), (160, 32768)]:
+        w = synth.t_weight(rows, cols, nu=4, scale=0.02, seed=rows + cols, device=DEV).cpu()
+        masks = synth.sign_masks(cols, seed=rows)
+        mxfp4_parity(w, masks, rows_sample=[0, rows - 1])
+        nv, mx = fq.quantize_dual(w.to(DEV), sign_masks=torch.from_numpy(masks.view(np.int32)).to(DEV))
+        torch.cuda.synchronize()
+        assert fq.check_status(nv.status) == 0
+        m = oracle.mxfp4_quant(np.ascontiguousarray(w[-1:].float().numpy()), sign_masks=masks)
+        _assert_eq("dual mx codes", _np(mx.codes)[-1:], m["codes"])
