@@ -1020,6 +1020,8 @@ def build_parser() -> argparse.ArgumentParser:
                          "calls: two launches per weight (fp4q_mxfp4_quant_absmax + the NVFP4 sweep); "
                          "groups: fp4q_mxfp4_quant_group + fp4q_nvfp4_sweep_group per --group weights")
     ap.add_argument("--group", type=int, default=4, help="weights per grouped launch (at most 32)")
+    ap.add_argument("--prio", default="none", choices=["none", "nv", "mx"],
+                    help="give the NVFP4 (nv) or the MXFP4 (mx) stream the higher CUDA stream priority")
     ap.add_argument("--layer-groups", default="",
                     help="split each layer's 7 weights (q,k,v,o,gate,up,down) into consecutive groups "
                          "of these sizes, e.g. 3,2,1,1 (overrides --group)")
@@ -1062,8 +1064,13 @@ def main():
     torch.cuda.set_device(dev)
 
     model = Model(fq, dev, seed=rank_seed(rank), with_events=True)
-    stream = torch.cuda.Stream(device=dev)
-    streams = [stream] + [torch.cuda.Stream(device=dev) for _ in range(args.streams - 1)]
+    p0 = p1 = 0
+    if args.prio != "none":
+        lo, hi = torch.cuda.Stream.priority_range()     # (least, greatest)
+        p0 = hi if args.prio == "mx" else lo             # stream 0 carries the MXFP4 launches
+        p1 = hi if args.prio == "nv" else lo             # the others the NVFP4 sweeps
+    stream = torch.cuda.Stream(device=dev, priority=p0)
+    streams = [stream] + [torch.cuda.Stream(device=dev, priority=p1) for _ in range(args.streams - 1)]
     stream.wait_stream(torch.cuda.current_stream())
     graph = torch.cuda.CUDAGraph()
 
