@@ -15,7 +15,8 @@
 // One thread owns one block: the rotation (sign flips, five in-register
 // butterfly stages h = 1..16, the 1/sqrt(32) multiply) and the sequential loss
 // stay in registers.  The three exponents are selected by screen-then-verify
-// (screen.cuh) in units of 2^e0, each exponent two elements at a time.  The Hadamard runs on the CUDA cores:
+// (screen.cuh) in units of 2^e0, each exponent two elements at a time (e0+1
+// is never the first minimum and is not screened, see kMxScreened).  The Hadamard runs on the CUDA cores:
 // it has to reproduce the stage order bit for bit, which a tensor-core
 // contraction does not, and it costs 6 adds/multiplies per element against a
 // memory budget of ~4.5 bytes per element.
@@ -27,6 +28,19 @@
 namespace fp4q {
 
 constexpr float kInvSqrt32 = 0x1.6a09e6p-3f;   // RN(1/sqrt(32))
+
+// Candidates screened: e0-1 and e0 only.  e0 is the smallest exponent whose
+// grid 2^e0 * {0, .5, 1, 1.5, 2, 3, 4, 6} covers the block maximum, and the
+// grid of e0+1 inside [0, 6 * 2^e0] is {0, 1, 2, 3, 4, 6} * 2^e0, a subset of
+// it: the nearest point of e0+1 is never nearer than that of e0, for every
+// element.  With power-of-two steps r = x * 2^-e and y = q * 2^e are exact
+// (an element too small for that has q = 0 under both), and RN(x - y),
+// RN(e * e) and the running sum are monotone, so the definition's loss at
+// e0+1 is never below the loss at e0 and the first minimum is never e0+1
+// (after clamping at 127 the two are the same exponent).  Its screened loss is
+// set to +inf: it survives only when the threshold is infinite, and then the
+// exact verification decides, as for any candidate.
+constexpr int kMxScreened = 2;
 
 // The 32 bf16 elements of a block from its 64 raw bytes, and max|w| as bits.
 __device__ __forceinline__ void unpack32_bf16_amax(const uint4* u, float (&x)[32], uint32_t& wmax)
@@ -105,10 +119,10 @@ __device__ __forceinline__ uint32_t mxfp4_block_pairs_of_neighbours(const T* __r
     const float tS = 0x1p-70f * inv0;
     const float tau = tS * tS + 0x1p-120f;
     float lam[3];
-    {   // the three exponents, two elements at a time
-        uint64_t inv2[3], L2[3];
+    {   // e0-1 and e0, two elements at a time; e0+1 never wins (kMxScreened)
+        uint64_t inv2[kMxScreened], L2[kMxScreened];
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
+        for (int k = 0; k < kMxScreened; ++k) {
             const float ik = exp2i(-FP4Q_EK(k));
             inv2[k] = pk(ik, ik);
             L2[k] = pk(0.0f, 0.0f);
@@ -117,7 +131,7 @@ __device__ __forceinline__ uint32_t mxfp4_block_pairs_of_neighbours(const T* __r
         for (int j = 0; j < 16; ++j) {
             const uint64_t xp = pk(x[2 * j], x[2 * j + 1]);
 #pragma unroll
-            for (int k = 0; k < 3; ++k) {
+            for (int k = 0; k < kMxScreened; ++k) {
                 float ra, rb;
                 upk(mul2(xp, inv2[k]), ra, rb);
                 const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
@@ -125,11 +139,12 @@ __device__ __forceinline__ uint32_t mxfp4_block_pairs_of_neighbours(const T* __r
             }
         }
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
+        for (int k = 0; k < kMxScreened; ++k) {
             float lo, hi;
             upk(L2[k], lo, hi);
             lam[k] = (lo + hi) * exp2i(2 * (FP4Q_EK(k) - e0));
         }
+        lam[2] = __int_as_float(0x7F800000);
     }
     const float M = fminf(fminf(lam[0], lam[1]), lam[2]);
     const float thr = survivor_threshold(M, alpha2, tau);
@@ -281,10 +296,10 @@ __device__ __forceinline__ uint32_t mxfp4_block_pairs_of_halves(const T* __restr
     const float tS = 0x1p-70f * inv0;
     const float tau = tS * tS + 0x1p-120f;
     float lam[3];
-    {   // the three exponents, one register pair at a time
-        uint64_t inv2[3], L2[3];
+    {   // e0-1 and e0, one register pair at a time; e0+1 never wins (kMxScreened)
+        uint64_t inv2[kMxScreened], L2[kMxScreened];
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
+        for (int k = 0; k < kMxScreened; ++k) {
             const float ik = exp2i(-FP4Q_EK(k));
             inv2[k] = pk(ik, ik);
             L2[k] = pk(0.0f, 0.0f);
@@ -292,7 +307,7 @@ __device__ __forceinline__ uint32_t mxfp4_block_pairs_of_halves(const T* __restr
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
 #pragma unroll
-            for (int k = 0; k < 3; ++k) {
+            for (int k = 0; k < kMxScreened; ++k) {
                 float ra, rb;
                 upk(mul2(P[j], inv2[k]), ra, rb);
                 const uint64_t et = sub_h2_f2(e2m1x2_round_h(ra, rb), ra, rb);
@@ -300,11 +315,12 @@ __device__ __forceinline__ uint32_t mxfp4_block_pairs_of_halves(const T* __restr
             }
         }
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
+        for (int k = 0; k < kMxScreened; ++k) {
             float lo, hi;
             upk(L2[k], lo, hi);
             lam[k] = (lo + hi) * exp2i(2 * (FP4Q_EK(k) - e0));
         }
+        lam[2] = __int_as_float(0x7F800000);
     }
     const float M = fminf(fminf(lam[0], lam[1]), lam[2]);
     const float thr = survivor_threshold(M, alpha2, tau);

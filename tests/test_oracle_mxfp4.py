@@ -283,3 +283,53 @@ def test_cutlass_atom_constants_match_the_header():
     assert "usingSfKMajorAtom=Layout<Shape<Shape<_32,_4>,Shape<Int<SFVecSize>,_4>>," in text
     assert "Stride<Stride<_16,_4>,Stride<_0,_1>>>;" in text
     assert "tile_to_shape(SfAtom{},make_shape(M,K),Step<_2,_1>{})" in text
+
+
+def _centre(xb):
+    import oracle
+    return np.array([oracle.mx_centre_exponent(a) for a in np.abs(xb).max(axis=1)])
+
+
+@pytest.mark.parametrize("kind", ["t3", "t4", "uniform", "ties", "huge", "tiny", "rotated"])
+def test_mxfp4_never_picks_the_exponent_above_the_centre(orc, kind):
+    """E8M0 steps are powers of two and e0 is the smallest exponent whose grid
+    covers the block maximum, so the grid of e0+1 restricted to the block's
+    range is a subset of the grid of e0: every element's error at e0+1 is at
+    least its error at e0, every product and quotient is exact in binary32
+    (powers of two), and each rounding step of the loss is monotone, so the
+    loss at e0+1 is never below the loss at e0 and the first minimum is never
+    e0+1 (the kernels skip screening it).  Checked on the oracle's choice over
+    heavy-tailed, uniform, tie-only, near-overflow, subnormal and rotated
+    blocks, and in fp64 against the e0 loss."""
+    rng = np.random.default_rng(40 + len(kind))
+    masks = None
+    if kind in ("t3", "t4"):
+        x = synth.t_weight(64, 1024, nu=int(kind[1]), scale=0.02, seed=41).float().numpy()
+    elif kind == "uniform":
+        x = rng.uniform(-1, 1, size=(64, 1024)).astype(np.float32)
+    elif kind == "ties":
+        # every element on a midpoint of the e0 grid (the equal-loss edge), plus the block maximum 6 * 2^k
+        mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+        g = mids[rng.integers(0, len(mids), size=(2048, 32))] * np.where(rng.random((2048, 32)) < .5, -1, 1)
+        g[:, 7] = 6.0
+        x = (g * 2.0 ** rng.integers(-20, 20, size=(2048, 1))).astype(np.float32).reshape(64, 1024)
+    elif kind == "huge":
+        x = (rng.uniform(-1, 1, size=(64, 1024)) * 3.0e38).astype(np.float32)
+    elif kind == "tiny":
+        x = (rng.uniform(-1, 1, size=(64, 1024)) * 2.0 ** -126).astype(np.float32)
+    else:
+        x = synth.t_weight(64, 1024, nu=3, scale=0.015, seed=42).float().numpy()
+        masks = synth.sign_masks(1024, seed=42)
+    out = orc.mxfp4_quant(x, sign_masks=masks)
+    if kind != "huge":
+        assert out["status"] == 0
+    vb = (out["rotated"] if masks is not None else x).reshape(-1, 32)
+    e0 = _centre(vb)
+    chosen = out["scales"].reshape(-1).astype(np.int64) - 127
+    above = np.minimum(e0 + 1, 127)
+    assert np.all((chosen != above) | (above == e0)), "e0+1 chosen"
+    if kind not in ("huge", "tiny"):
+        d = np.exp2(np.stack([e0, e0 + 1], 1).astype(np.float64)).astype(np.float32)
+        inv = np.exp2(-np.stack([e0, e0 + 1], 1).astype(np.float64)).astype(np.float32)
+        loss64, _, _ = block_losses(vb, d, inv)
+        assert np.all(loss64[:, 1] >= loss64[:, 0])
