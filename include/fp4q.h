@@ -308,7 +308,10 @@ size_t fp4q_gptq_workspace_bytes(int64_t rows);
  * The blocked GPU algorithm applies these updates to every element in the
  * same order, so its bytes are those of the sequential definition.
  *   w          device fp32 rows x cols (cols % 16 == 0), 16-byte aligned;
- *              OVERWRITTEN with the error-compensated values.
+ *              used as scratch and OVERWRITTEN: each 128-column block is
+ *              left holding its values after the updates of the blocks
+ *              before it (the updates inside the block stay in registers),
+ *              so keep a copy if the original weight is needed.
  *   U          device fp32 cols x cols, row-major; only the upper triangle
  *              (diagonal included) is read.
  *   d_amax     device float: max|w| of the original weight
