@@ -60,10 +60,13 @@ struct MxGroupParams {
 };
 
 // The thread block's item sits in shared memory and its pointers are read
-// there (volatile, so not hoisted into registers) at every block: held in
-// registers across the loop they push the 64-register kernel into spills.
+// there (volatile, so not hoisted into registers) at every block.  Three
+// thread blocks per SM, not the single-weight kernel's four: the grouped
+// MXFP4 launch runs beside the NVFP4 sweep of the previous group, and fewer
+// resident MXFP4 warps leave room for the sweep (whole-model step 18.33/18.25
+// -> 17.93/17.90 ms on one box; two blocks per SM: 18.74 ms).
 template <typename T, bool HAD>
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kThreads, 3)
 mxfp4_group_kernel(const __grid_constant__ MxGroupParams P, int32_t* __restrict__ d_status, float neg_zero)
 {
     __shared__ MxGroupParams::Item item;
