@@ -162,6 +162,27 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- workload
 
+def group_bounds(n, size, layer_sizes=None):
+    """[lo, hi) index ranges of the grouped launches over n weights: consecutive
+    groups of `size`, or each layer's weights (sum(layer_sizes) of them) split
+    into consecutive groups of layer_sizes.  Every weight is in exactly one
+    range, in order."""
+    if layer_sizes:
+        if min(layer_sizes) < 1:
+            raise ValueError("group sizes must be positive")
+        per_layer = sum(layer_sizes)
+        bounds = []
+        for base in range(0, n, per_layer):
+            for k in layer_sizes:
+                if base < n:
+                    bounds.append((base, min(base + k, n)))
+                base += k
+        return bounds
+    if size < 1:
+        raise ValueError("group size must be positive")
+    return [(b, min(b + size, n)) for b in range(0, n, size)]
+
+
 class Model:
     """Device buffers of the whole-model pass and the launch sequence of one step."""
 
@@ -220,16 +241,7 @@ class Model:
         consecutive weights in groups of `size` (7 = one layer), or each layer's seven
         weights split into consecutive groups of `layer_sizes` (summing to 7)."""
         self.groups = []
-        if layer_sizes:
-            per_layer = sum(layer_sizes)
-            bounds = []
-            for base in range(0, len(self.w), per_layer):
-                for k in layer_sizes:
-                    bounds.append((base, min(base + k, len(self.w))))
-                    base += k
-        else:
-            bounds = [(b, min(b + size, len(self.w))) for b in range(0, len(self.w), size)]
-        for lo, hi in bounds:
+        for lo, hi in group_bounds(len(self.w), size, layer_sizes):
             idx = range(lo, hi)
             mx = [dict(w=self.w[i], amax=self.out[i]["amax"], mx_codes=self.out[i]["mx_codes"],
                        mx_scales=self.out[i]["mx_scales"], mx_deq=self.out[i]["mx_deq"]) for i in idx]

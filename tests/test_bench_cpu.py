@@ -41,3 +41,29 @@ def test_profile_commands_use_existing_benchmark_options():
     for path, tail in cmds:
         args = shlex.split(tail.split(">")[0])
         parser.parse_args(args)          # SystemExit on an unknown option or kernel name
+
+
+def test_group_bounds_cover_every_weight_once_in_order():
+    for n, size, layers in [(224, 4, None), (224, 3, None), (224, 7, None), (10, 32, None), (224, 1, None),
+                            (224, 0, [4, 1, 1, 1]), (224, 0, [3, 2, 2]), (23, 0, [3, 2, 2]), (7, 0, [7])]:
+        b = bench.group_bounds(n, size, layers)
+        covered = [i for lo, hi in b for i in range(lo, hi)]
+        assert covered == list(range(n)), (n, size, layers)
+        assert all(hi > lo for lo, hi in b)
+        if layers is None:
+            assert all(hi - lo <= size for lo, hi in b)
+            assert len(b) == -(-n // size)
+        else:
+            per = sum(layers)
+            # the groups repeat the layer pattern
+            sizes = [hi - lo for lo, hi in b]
+            assert sizes[:len(layers)] == [min(k, n) for k in layers][:len(sizes[:len(layers)])]
+            assert len(b) == len(layers) * (n // per) + len([k for k in np.cumsum([0] + layers[:-1]) if k < n % per])
+
+
+def test_group_bounds_reject_empty_groups():
+    import pytest
+    with pytest.raises(ValueError):
+        bench.group_bounds(10, 0)
+    with pytest.raises(ValueError):
+        bench.group_bounds(10, 4, [3, 0, 4])
