@@ -13,6 +13,9 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// One weight.  AMAX: also reduce max|w| of the unrotated input into
+// *gmax_bits (an atomic max on the binary32 bit pattern, which keeps NaN and
+// Inf), for the NVFP4 global scale of the same weight.
 template <typename T, bool HAD, bool AMAX>
 __global__ void __launch_bounds__(kThreads, 4)
 mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
