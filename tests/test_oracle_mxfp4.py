@@ -333,3 +333,30 @@ def test_mxfp4_never_picks_the_exponent_above_the_centre(orc, kind):
         inv = np.exp2(-np.stack([e0, e0 + 1], 1).astype(np.float64)).astype(np.float32)
         loss64, _, _ = block_losses(vb, d, inv)
         assert np.all(loss64[:, 1] >= loss64[:, 0])
+
+
+@pytest.mark.parametrize("e0", [-127, -126, -100, -3, 0, 5, 100, 126])
+def test_mxfp4_element_error_is_never_smaller_above_the_centre(e0):
+    """The lemma behind skipping e0+1, element by element and exhaustively:
+    for every positive finite bf16 value x (the sign is symmetric) with
+    x <= 6 * 2^e0, the definition's binary32 error term RN(RN(x - y)^2),
+    y = RN(q * 2^e), q the E2M1 point nearest to RN(x * 2^-e) (fp64 search,
+    ties to the even code), is at least as large at e = e0+1 as at e = e0."""
+    from fp64_check import e2m1_nearest
+    x = (np.arange(1, 0x7F80, dtype=np.uint32) << 16).view(np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        lim = np.float32(6.0) * np.float32(2.0 ** e0)
+        x = x[x <= lim]
+
+        def term(e):
+            d = np.float32(2.0 ** e)
+            inv = np.float32(2.0 ** -e)
+            r = (x * inv).astype(np.float32)
+            _, q = e2m1_nearest(r)
+            y = (q * np.float64(d)).astype(np.float32)
+            err = (x - y).astype(np.float32)
+            return (err * err).astype(np.float32)
+
+        t0, t1 = term(e0), term(e0 + 1)
+    assert x.size >= 300                       # 320 bf16 values even at the subnormal end
+    assert np.all(t1 >= t0)
