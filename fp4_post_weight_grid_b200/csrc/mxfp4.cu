@@ -48,6 +48,7 @@ mxfp4_kernel(const T* __restrict__ w, int64_t nblocks, int64_t blocks_per_row,
 
 // Several weights in one launch, each with the fused max: weight t owns
 // thread blocks [cta0, cta0 + nctas).
+constexpr int kMxGroupBlocksPerSm = 2;    // grid cap of the grouped launch
 struct MxGroupParams {
     int32_t n;
     struct Item {
@@ -110,7 +111,13 @@ void launch_group_typed(const GroupItem* items, int n, int32_t* d_status, cudaSt
     MxGroupParams P{};
     int64_t total = 0;
     for (int i = 0; i < n; ++i) total += items[i].rows * (items[i].cols / 32);
-    const int64_t rounds = grid_rounds(kernel, kThreads, 0, total);
+    // At most two thread blocks per SM over the whole launch (each takes more
+    // rounds), so that the pass stays beside the NVFP4 sweep for longer with
+    // fewer warps instead of filling the SMs and finishing early: whole-model
+    // step 17.84 -> 17.66-17.69 ms (one per SM: 20.8 ms).
+    int64_t rounds = grid_rounds(kernel, kThreads, 0, total);
+    const int64_t per_launch = (int64_t)kMxGroupBlocksPerSm * sm_count() * kThreads;
+    if ((total + per_launch - 1) / per_launch > rounds) rounds = (total + per_launch - 1) / per_launch;
     int64_t cta = 0;
     P.n = 0;
     for (int i = 0; i < n; ++i) {
